@@ -1,0 +1,215 @@
+"""Thin Python binding of the C ABI in include/topk_b200.h.
+
+Argument marshalling only: every step of the selection runs in the CUDA
+library (libtopk_b200.so).  PyTorch provides device memory and the current
+stream; there is no CPU fallback -- a missing library or a non-CUDA tensor is an
+error.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+TOPK_OK, TOPK_EINVAL, TOPK_EUNSUPPORTED, TOPK_ECUDA, TOPK_EWORKSPACE = range(5)
+TOPK_OP_BUCKETED, TOPK_OP_EXACT, TOPK_OP_SCORE = range(3)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class TopkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s" % (where, topk_status_string(status)))
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library():
+    """Load libtopk_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if not os.path.exists(path):
+                raise ImportError(
+                    "libtopk_b200.so is missing: build it with "
+                    "`python -m approximate_top_selection_b200.build`")
+            lib = ctypes.CDLL(path)
+            i64, i32, p, sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+            lib.topk_workspace_bytes.argtypes = [i32, i64, i64, i32, i32, i32, i32]
+            lib.topk_workspace_bytes.restype = sz
+            lib.topk_bucketed.argtypes = [p, i64, i64, i32, i32, i32, p, p, p, sz, p]
+            lib.topk_bucketed.restype = i32
+            lib.topk_exact.argtypes = [p, i64, i64, i32, p, p, p, sz, p]
+            lib.topk_exact.restype = i32
+            lib.score_topk.argtypes = [p, i64, i32, p, i64, i64, i32, i32, i32, p, p, p, p, sz, p]
+            lib.score_topk.restype = i32
+            lib.topk_status_string.argtypes = [i32]
+            lib.topk_status_string.restype = ctypes.c_char_p
+            lib.topk_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
+            lib.topk_device_status.restype = i32
+            _lib = lib
+    return _lib
+
+
+def topk_status_string(status: int) -> str:
+    return load_library().topk_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != TOPK_OK:
+        raise TopkError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtype) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+# One zero-filled workspace per (device, stream); every call leaves it zeroed.
+_ws_cache: dict = {}
+
+
+def _workspace(nbytes: int, device: torch.device, stream: int) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    key = (device.index, stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+_ws_bytes_cache: dict = {}
+
+
+def topk_workspace_bytes(op: int, rows: int, n: int, k: int, b: int = 1, kb: int = 1,
+                         d: int = 0) -> int:
+    """Workspace bytes of a call on the current device (cached per shape)."""
+    key = (torch.cuda.current_device(), op, rows, n, k, b, kb, d)
+    v = _ws_bytes_cache.get(key)
+    if v is None:
+        v = int(load_library().topk_workspace_bytes(op, rows, n, k, b, kb, d))
+        _ws_bytes_cache[key] = v
+    return v
+
+
+def _outputs(rows: int, k: int, device, out_vals, out_idx):
+    if out_vals is None:
+        out_vals = torch.empty(rows, k, dtype=torch.float32, device=device)
+    if out_idx is None:
+        out_idx = torch.empty(rows, k, dtype=torch.int32, device=device)
+    _cuda(out_vals, "out_vals", torch.float32)
+    _cuda(out_idx, "out_idx", torch.int32)
+    if out_vals.numel() != rows * k or out_idx.numel() != rows * k:
+        raise ValueError("outputs must hold rows*k elements")
+    return out_vals, out_idx
+
+
+def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=None, out_idx=None,
+                  workspace: torch.Tensor | None = None, stream=None):
+    """Bucketed approximate top-k of every row of `scores` ([rows, n] float32, CUDA).
+
+    Returns (values [rows, k] float32, indices [rows, k] int32), best-first,
+    padded with -inf / -1.
+    """
+    lib = load_library()
+    _cuda(scores, "scores", torch.float32)
+    if scores.dim() != 2:
+        raise ValueError("scores must be [rows, n]")
+    rows, n = scores.shape
+    with torch.cuda.device(scores.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
+        need = topk_workspace_bytes(TOPK_OP_BUCKETED, rows, n, k, b, kb)
+        ws = workspace if workspace is not None else _workspace(need, scores.device, sh)
+        st = lib.topk_bucketed(scores.data_ptr(), rows, n, k, b, kb, out_vals.data_ptr(),
+                               out_idx.data_ptr(), ws.data_ptr() if ws is not None else None,
+                               ws.numel() if ws is not None else 0, sh)
+    _check(st, "topk_bucketed")
+    return out_vals, out_idx
+
+
+def topk_exact(scores: torch.Tensor, k: int, *, out_vals=None, out_idx=None, stream=None):
+    """Exact top-k of every row (ties by lowest index), padded with -inf / -1."""
+    lib = load_library()
+    _cuda(scores, "scores", torch.float32)
+    if scores.dim() != 2:
+        raise ValueError("scores must be [rows, n]")
+    rows, n = scores.shape
+    with torch.cuda.device(scores.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
+        st = lib.topk_exact(scores.data_ptr(), rows, n, k, out_vals.data_ptr(),
+                            out_idx.data_ptr(), None, 0, sh)
+    _check(st, "topk_exact")
+    return out_vals, out_idx
+
+
+def score_topk(q: torch.Tensor, K: torch.Tensor, k: int, b: int, kb: int, *,
+               return_scores: bool = False, out_vals=None, out_idx=None,
+               workspace: torch.Tensor | None = None, stream=None):
+    """Fused q.K scoring and bucketed top-k.
+
+    q: [rows, d] bfloat16.  K: [rows, n, d] (one key matrix per row) or [n, d]
+    (shared by all rows), bfloat16.  Returns (values, indices[, scores]).
+    """
+    lib = load_library()
+    _cuda(q, "q", torch.bfloat16)
+    _cuda(K, "K", torch.bfloat16)
+    if q.dim() != 2:
+        raise ValueError("q must be [rows, d]")
+    rows, d = q.shape
+    if K.dim() == 3:
+        if K.shape[0] != rows:
+            raise ValueError("K must be [rows, n, d] or [n, d]")
+        n, stride = K.shape[1], K.shape[1] * d
+    elif K.dim() == 2:
+        n, stride = K.shape[0], 0
+    else:
+        raise ValueError("K must be [rows, n, d] or [n, d]")
+    if K.shape[-1] != d:
+        raise ValueError("q and K disagree on d")
+    with torch.cuda.device(q.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
+        scores = torch.empty(rows, n, dtype=torch.float32, device=q.device) if return_scores else None
+        need = topk_workspace_bytes(TOPK_OP_SCORE, rows, n, k, b, kb, d)
+        ws = workspace if workspace is not None else _workspace(need, q.device, sh)
+        st = lib.score_topk(q.data_ptr(), rows, d, K.data_ptr(), n, stride, k, b, kb,
+                            out_vals.data_ptr(), out_idx.data_ptr(),
+                            scores.data_ptr() if scores is not None else None,
+                            ws.data_ptr() if ws is not None else None,
+                            ws.numel() if ws is not None else 0, sh)
+    _check(st, "score_topk")
+    if return_scores:
+        return out_vals, out_idx, scores
+    return out_vals, out_idx
+
+
+def topk_device_status() -> int:
+    """Read and clear the device status word (synchronises the device)."""
+    v = ctypes.c_int(0)
+    _check(load_library().topk_device_status(ctypes.byref(v)), "topk_device_status")
+    return int(v.value)

@@ -1,0 +1,239 @@
+// bucket_select.cuh -- Stage 1 + Stage 2 of bucketed top-k over float32 rows.
+//
+// Method: "Approximate Top-k for Increased Parallelism" (arXiv 2412.04358),
+// pith.science review page, "What carries the argument": interleaved buckets
+// (element i -> bucket i mod b), exact top-k_b per bucket kept in per-thread
+// register queues (k_b <= 4), final exact top-k when b*k_b > k.
+//
+// Work decomposition (ours, not the page's): the rows*n elements are cut into
+// G equal contiguous CTA ranges, so every CTA streams the same number of bytes
+// whatever the row count; a row that straddles CTA ranges is merged by the last
+// CTA to finish it (select_core.cuh).
+//
+// Fast kernel (n % 4 == 0, 16-byte aligned rows, b | 1024): the TMA engine
+// streams 16 KB tiles of the row into a ring of shared-memory stages
+// (cp.async.bulk + mbarrier); thread t owns the four consecutive positions
+// 4t..4t+3 of every 1024-element stripe, so each of its four queues sees a
+// single bucket ((a + 4t + v) mod b) and needs no communication until the end.
+// General kernel (any n, alignment, b <= 1024): direct coalesced scalar loads,
+// thread t owns stripe positions t + 256 v of a stripe of L*b elements.
+#pragma once
+
+#include "select_core.cuh"
+
+namespace tk {
+
+constexpr int kTile = 4096;  // floats per bulk copy (16 KB)
+
+struct SelectArgs {
+  const float* x;
+  int k, b;
+  float* out_vals;
+  int32_t* out_idx;
+  RowSplit rs;
+};
+
+// Shared-memory layout of the selection kernels (bytes).
+struct SelectSmem {
+  int stages, kb, cand_cap;
+  __host__ __device__ size_t ring_bytes() const { return static_cast<size_t>(stages) * kTile * 4; }
+  __host__ __device__ size_t lane_bytes() const { return static_cast<size_t>(kLanes) * kb * 8; }
+  __host__ __device__ size_t cand_bytes() const { return static_cast<size_t>(cand_cap) * 8; }
+  __host__ __device__ size_t bar_bytes() const { return 16 * static_cast<size_t>(stages) + 16; }
+  __host__ __device__ size_t total() const {
+    return ring_bytes() + lane_bytes() + cand_bytes() + bar_bytes();
+  }
+};
+
+constexpr int kConsumerWarps = kThreads / 32;
+constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
+
+// Warp-specialised streaming: warp kConsumerWarps issues the bulk copies of
+// the CTA's tiles into a ring of `stages` shared-memory stages (full barrier:
+// bytes landed; empty barrier: every consumer warp is done with the stage);
+// the kThreads consumer threads never wait for each other inside a piece.
+template <int KB>
+__global__ void __launch_bounds__(kPipeThreads) bucket_select_tma(SelectArgs p, int stages,
+                                                                  int cand_cap) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SelectSmem L{stages, KB, cand_cap};
+  float* ring = reinterpret_cast<float*>(smem);
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes() + L.cand_bytes());
+  uint64_t* empty = full + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  int* piece_flag = reinterpret_cast<int*>(empty + stages) + 1;
+
+  const RowSplit& rs = p.rs;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t s0 = cta_start(rs, blockIdx.x);
+  const int64_t e0 = cta_start(rs, blockIdx.x + 1);
+  const int64_t n = rs.n;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // Tile t of this CTA covers [g, g + len) with len = min(kTile, e0 - g,
+  // end of g's row - g): tiles never straddle rows.
+  auto tile_len = [&](int64_t g) -> int64_t {
+    const int64_t rowend = (g / n + 1) * n;
+    int64_t c = e0 - g;
+    if (rowend - g < c) c = rowend - g;
+    return c < kTile ? c : kTile;
+  };
+
+  if (warp == kConsumerWarps) {  // ---------------- producer
+    if (lane == 0) {
+      int64_t g = s0, t = 0;
+      int st = 0;       // stage of tile t
+      uint32_t ph = 0;  // parity of t / stages
+      while (g < e0) {
+        const int64_t c = tile_len(g);
+        if (t >= stages && !mbar_wait_or_abort(empty + st, ph ^ 1u, abort_flag)) break;
+        const uint32_t bytes = static_cast<uint32_t>(c * 4);
+        mbar_expect_tx(full + st, bytes);
+        bulk_g2s(ring + static_cast<size_t>(st) * kTile, p.x + g, bytes, full + st);
+        g += c;
+        ++t;
+        if (++st == stages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA can go away.
+        for (int64_t u = (t > stages ? t - stages : 0); u < t; ++u)
+          mbar_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), 100000000ull);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers
+  Queues<KB> q;
+  int st = 0;       // ring stage of the next tile
+  uint32_t ph = 0;  // its full-barrier parity
+  int64_t g = s0;
+  while (g < e0) {
+    const int64_t r = g / n;
+    const int64_t row0 = r * n;
+    const int64_t a = g - row0;
+    const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
+    q.reset();
+    while (g < pend) {
+
+      const int64_t c = (pend - g) < kTile ? (pend - g) : kTile;
+      // Warp-uniform: if any lane saw the stage complete, its bytes have landed.
+      const bool ok = __any_sync(0xffffffffu,
+                                 !*abort_flag &&
+                                     mbar_wait_or_abort(full + st, ph, abort_flag));
+      if (ok) {
+        const float* tile = ring + static_cast<size_t>(st) * kTile;
+        const uint32_t pos0 = static_cast<uint32_t>(g - row0);
+        constexpr int U = kTile / kLanes;
+        float4 x[U];
+        uint32_t i0[U];
+        bool valid[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int off = 4 * tid + kLanes * u;
+          valid[u] = off < c;
+          x[u] = valid[u] ? *reinterpret_cast<const float4*>(tile + off)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+          i0[u] = pos0 + static_cast<uint32_t>(off);
+        }
+        q.template offer_rows<U>(x, i0, valid);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + st);
+      if (++st == stages) {
+        st = 0;
+        ph ^= 1u;
+      }
+      g += c;
+    }
+    // Piece done: publish the queues and finish (Stage 2 or cross-CTA merge).
+#pragma unroll
+    for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
+    group_sync(kThreads);
+    finish_piece<KB, kGatherInput>(rs, p.b, p.k, r, a, pend - row0 - a, lanebuf, cand,
+                                   p.x + row0, p.out_vals, p.out_idx, piece_flag);
+    group_sync(kThreads);
+  }
+}
+
+template <int KB>
+__global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, int cand_cap) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SelectSmem L{0, KB, cand_cap};
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.lane_bytes());
+  __shared__ int piece_flag;
+
+  const RowSplit& rs = p.rs;
+  const int tid = threadIdx.x;
+  const int64_t s0 = cta_start(rs, blockIdx.x);
+  const int64_t e0 = cta_start(rs, blockIdx.x + 1);
+  const int64_t n = rs.n;
+  const int b = p.b;
+  const int W = (kLanes / b) * b;  // stripe: lanes per bucket times b
+
+  Queues<KB> q;
+  int64_t g = s0;
+  while (g < e0) {
+    const int64_t r = g / n;
+    const int64_t row0 = r * n;
+    const int64_t a = g - row0;
+    const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
+    const int64_t len = pend - g;
+    const float* src = p.x + g;
+    q.reset();
+    constexpr int U = 4;  // stripes in flight per thread
+    for (int64_t base = 0; base < len; base += static_cast<int64_t>(W) * U) {
+      float v[U][4];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int l = tid + kThreads * w;
+          const int64_t off = base + static_cast<int64_t>(W) * u + l;
+          v[u][w] = (l < W && off < len) ? __ldg(src + off) : __uint_as_float(0xff800000u);
+        }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int l = tid + kThreads * w;
+          const int64_t off = base + static_cast<int64_t>(W) * u + l;
+          if (l < W && off < len) {
+            const uint32_t pos = static_cast<uint32_t>(a + off);
+            if (w == 0) q.template offer<0>(v[u][0], pos);
+            if (w == 1) q.template offer<1>(v[u][1], pos);
+            if (w == 2) q.template offer<2>(v[u][2], pos);
+            if (w == 3) q.template offer<3>(v[u][3], pos);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      q.store(w, lanebuf + static_cast<size_t>(tid + kThreads * w) * KB);
+    group_sync(kThreads);
+    finish_piece<KB, kGatherInput>(rs, b, p.k, r, a, len, lanebuf, cand, p.x + row0, p.out_vals,
+                                   p.out_idx, &piece_flag);
+    group_sync(kThreads);
+    g = pend;
+  }
+}
+
+}  // namespace tk

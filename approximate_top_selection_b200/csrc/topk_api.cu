@@ -1,0 +1,470 @@
+// topk_api.cu -- the C ABI (include/topk_b200.h): argument checks, launch
+// plans and kernel launches.  All device work lives in the included kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/topk_b200.h"
+#include "bucket_select.cuh"
+#include "exact_topk.cuh"
+#include "score_gemv.cuh"
+
+namespace tk {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxN = 2147483647LL;       // indices are int32
+constexpr int64_t kMaxElems = 1LL << 50;      // keeps the partition arithmetic in int64
+constexpr int64_t kSelectMinPiece = 16384;    // elements per CTA before splitting pays
+constexpr int64_t kScoreMinPiece = 1024;      // keys per CTA
+
+// Ring depth: as many 16 KB stages as fit while kCtasPerSm CTAs share an SM's
+// shared memory (bytes in flight per SM are what keeps HBM busy), clamped.
+#ifndef TOPK_CTAS_PER_SM
+#define TOPK_CTAS_PER_SM 2
+#endif
+#ifndef TOPK_MAX_STAGES
+#define TOPK_MAX_STAGES 8
+#endif
+constexpr size_t kSmemPerSm = 228 * 1024;
+constexpr size_t kSmemReservedPerCta = 1024;
+
+template <typename Layout>
+int fit_stages(Layout L, int min_stages) {
+  const size_t budget = kSmemPerSm / TOPK_CTAS_PER_SM - kSmemReservedPerCta;
+  int st = TOPK_MAX_STAGES;
+  for (; st > min_stages; --st) {
+    L.stages = st;
+    if (L.total() <= budget) break;
+  }
+  return st;
+}
+
+struct DeviceInfo {
+  bool init = false;
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int current_device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TOPK_ECUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return TOPK_ECUDA;
+    if (cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+      return TOPK_ECUDA;
+    d.init = true;
+  }
+  *out = d;
+  return TOPK_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int host_next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// Launch plan shared by topk_bucketed / score_topk and their workspace query.
+struct Plan {
+  int G = 0;
+  int align = 1;
+  int stages = 0;
+  int cand_cap = 0;
+  size_t smem = 0;
+  int64_t units = 0;
+  size_t ws_tickets = 0;  // bytes
+  size_t ws_slots = 0;    // bytes
+  size_t workspace() const { return ws_tickets + ws_slots; }
+};
+
+// Resident CTAs per SM of (kernel, dynamic smem) on a device, cached: the
+// attribute call and the occupancy query cost microseconds of host time.
+struct OccKey {
+  int dev;
+  const void* fn;
+  size_t smem;
+  int blocks;
+};
+constexpr int kOccSlots = 256;
+OccKey g_occ[kOccSlots];
+int g_occ_n = 0;
+std::mutex g_occ_mu;
+
+// Kernels whose dynamic shared-memory limit has been raised, per device.  The
+// limit is raised once to the device's opt-in maximum, so any later launch of
+// the kernel may use any size up to it (a per-size setting would be undone by
+// the next call that asks for less).
+struct AttrKey {
+  int dev;
+  const void* fn;
+};
+AttrKey g_attr[kOccSlots];
+int g_attr_n = 0;
+
+template <typename KernelT>
+int raise_smem_limit_locked(KernelT kernel, int dev, int max_optin) {
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  for (int i = 0; i < g_attr_n; ++i)
+    if (g_attr[i].dev == dev && g_attr[i].fn == fn) return TOPK_OK;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return TOPK_ECUDA;
+  const int dyn_max = max_optin - static_cast<int>(fa.sharedSizeBytes);
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
+      cudaSuccess)
+    return TOPK_ECUDA;
+  if (g_attr_n >= kOccSlots) return TOPK_ECUDA;
+  g_attr[g_attr_n++] = AttrKey{dev, fn};
+  return TOPK_OK;
+}
+
+template <typename KernelT>
+int prepare_kernel(KernelT kernel) {
+  int dev = 0, max_optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TOPK_ECUDA;
+  if (cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+      cudaSuccess)
+    return TOPK_ECUDA;
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  return raise_smem_limit_locked(kernel, dev, max_optin);
+}
+
+template <typename KernelT>
+int occupancy(KernelT kernel, int block, size_t smem, int* blocks) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TOPK_ECUDA;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  {
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    for (int i = 0; i < g_occ_n; ++i) {
+      if (g_occ[i].dev == dev && g_occ[i].fn == fn && g_occ[i].smem == smem) {
+        *blocks = g_occ[i].blocks;
+        return TOPK_OK;
+      }
+    }
+  }
+  int rc = prepare_kernel(kernel);
+  if (rc) return rc;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, kernel, block, smem) != cudaSuccess)
+    return TOPK_ECUDA;
+  if (*blocks < 1) return TOPK_EUNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_occ_mu);
+  if (g_occ_n < kOccSlots) g_occ[g_occ_n++] = OccKey{dev, fn, smem, *blocks};
+  return TOPK_OK;
+}
+
+// Number of CTAs: one per row when the rows alone fill the GPU and fit in one
+// resident wave (no row is split); otherwise the flattened element space is cut
+// into equal ranges, as many as fit in one wave, but no smaller than min_piece.
+int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, int per_sm) {
+  const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+  const int64_t units = E / align;
+  int64_t G;
+  if (rows <= cap && (rows >= sms || rows * min_piece >= E)) {
+    G = rows;  // one row per CTA: no row is split
+  } else {
+    G = std::min<int64_t>(cap, std::max<int64_t>(1, (E + min_piece - 1) / min_piece));
+    G = std::max<int64_t>(G, std::min<int64_t>(rows, cap));
+  }
+  G = std::max<int64_t>(1, std::min<int64_t>(G, units));
+  return static_cast<int>(G);
+}
+
+template <int KB>
+int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
+  const int C = b * KB;
+  pl->cand_cap = host_next_pow2(C);
+  pl->align = fast ? 4 : 1;
+  pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap}, 2) : 0;
+  int per_sm = 0;
+  if (fast) {
+    SelectSmem L{pl->stages, KB, pl->cand_cap};
+    pl->smem = L.total();
+    if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+    int rc = occupancy(bucket_select_tma<KB>, kPipeThreads, pl->smem, &per_sm);
+    if (rc) return rc;
+  } else {
+    SelectSmem L{0, KB, pl->cand_cap};
+    pl->smem = L.total();
+    if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+    int rc = occupancy(bucket_select_general<KB>, kThreads, pl->smem, &per_sm);
+    if (rc) return rc;
+  }
+  const int64_t E = rows * n;
+  pl->G = choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm);
+  pl->units = E / pl->align;
+  pl->ws_tickets = align_up(static_cast<size_t>(rows) * 4, 256);
+  pl->ws_slots = static_cast<size_t>(pl->G) * 2 * C * 8;
+  return TOPK_OK;
+}
+
+int plan_select(bool fast, int64_t rows, int64_t n, int b, int kb, const DeviceInfo& dev,
+                Plan* pl) {
+  switch (kb) {
+    case 1: return plan_select_kb<1>(fast, rows, n, b, dev, pl);
+    case 2: return plan_select_kb<2>(fast, rows, n, b, dev, pl);
+    case 3: return plan_select_kb<3>(fast, rows, n, b, dev, pl);
+    case 4: return plan_select_kb<4>(fast, rows, n, b, dev, pl);
+  }
+  return TOPK_EINVAL;
+}
+
+template <int KB, int D>
+int plan_score_kd(int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
+  const int C = b * KB;
+  pl->cand_cap = host_next_pow2(C);
+  pl->align = 1;
+  pl->stages = fit_stages(ScoreSmem{0, KB, pl->cand_cap}, 2);
+  ScoreSmem L{pl->stages, KB, pl->cand_cap};
+  pl->smem = L.total();
+  if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  int per_sm = 0;
+  int rc = occupancy(score_select_gemv<KB, D>, kScorePipeThreads, pl->smem, &per_sm);
+  if (rc) return rc;
+  const int64_t E = rows * n;
+  pl->G = choose_grid(rows, E, 1, kScoreMinPiece, dev.sms, per_sm);
+  pl->units = E;
+  pl->ws_tickets = align_up(static_cast<size_t>(rows) * 4, 256);
+  pl->ws_slots = static_cast<size_t>(pl->G) * 2 * C * 8;
+  return TOPK_OK;
+}
+
+template <int KB>
+int plan_score_k(int64_t rows, int64_t n, int b, int d, const DeviceInfo& dev, Plan* pl) {
+  if (d == 128) return plan_score_kd<KB, 128>(rows, n, b, dev, pl);
+  if (d == 256) return plan_score_kd<KB, 256>(rows, n, b, dev, pl);
+  return TOPK_EUNSUPPORTED;
+}
+
+int plan_score(int64_t rows, int64_t n, int b, int kb, int d, const DeviceInfo& dev, Plan* pl) {
+  switch (kb) {
+    case 1: return plan_score_k<1>(rows, n, b, d, dev, pl);
+    case 2: return plan_score_k<2>(rows, n, b, d, dev, pl);
+    case 3: return plan_score_k<3>(rows, n, b, d, dev, pl);
+    case 4: return plan_score_k<4>(rows, n, b, d, dev, pl);
+  }
+  return TOPK_EINVAL;
+}
+
+int check_common(int64_t rows, int64_t n, int k, int b, int kb) {
+  if (rows < 1 || n < 1 || k < 1 || b < 1 || kb < 1 || kb > kMaxKb) return TOPK_EINVAL;
+  if (n > kMaxN) return TOPK_EINVAL;
+  if (rows > kMaxElems / n) return TOPK_EUNSUPPORTED;
+  if (b > kMaxB || k > kMaxK) return TOPK_EUNSUPPORTED;
+  return TOPK_OK;
+}
+
+bool select_fast(const float* x, int64_t n, int b) {
+  return aligned16(x) && (n % 4) == 0 && (kLanes % b) == 0;
+}
+
+RowSplit make_split(const Plan& pl, int64_t rows, int64_t n, void* ws) {
+  RowSplit rs;
+  rs.rows = rows;
+  rs.n = n;
+  rs.E = rows * n;
+  rs.units = pl.units;
+  rs.G = pl.G;
+  rs.align = pl.align;
+  rs.tickets = static_cast<uint32_t*>(ws);
+  rs.slots = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(ws) + pl.ws_tickets);
+  return rs;
+}
+
+// A row is split iff the plan gives it to more than one CTA; only then is the
+// workspace touched.  With G == rows and one row per CTA no workspace is needed.
+bool plan_needs_workspace(const Plan& pl, int64_t rows, int64_t n) {
+  if (pl.G == rows && pl.align == 1) return false;
+  if (pl.G == rows && (n % pl.align) == 0) return false;
+  return true;
+}
+
+// Launch errors are read right after the launch; a non-sticky error left by
+// an earlier, unrelated runtime call is cleared first (clear_launch_error) so
+// that it is not reported as this launch's failure.
+void clear_launch_error() { (void)cudaGetLastError(); }
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? TOPK_OK : TOPK_ECUDA;
+}
+
+template <int KB>
+int launch_select_kb(bool fast, const Plan& pl, const SelectArgs& a, cudaStream_t st) {
+  clear_launch_error();
+  if (fast)
+    bucket_select_tma<KB><<<pl.G, kPipeThreads, pl.smem, st>>>(a, pl.stages, pl.cand_cap);
+  else
+    bucket_select_general<KB><<<pl.G, kThreads, pl.smem, st>>>(a, pl.cand_cap);
+  return launch_status();
+}
+
+template <int KB, int D>
+int launch_score_kd(const Plan& pl, const ScoreArgs& a, cudaStream_t st) {
+  clear_launch_error();
+  score_select_gemv<KB, D><<<pl.G, kScorePipeThreads, pl.smem, st>>>(a, pl.stages, pl.cand_cap);
+  return launch_status();
+}
+
+template <int KB>
+int launch_score_k(int d, const Plan& pl, const ScoreArgs& a, cudaStream_t st) {
+  if (d == 128) return launch_score_kd<KB, 128>(pl, a, st);
+  return launch_score_kd<KB, 256>(pl, a, st);
+}
+
+}  // namespace
+}  // namespace tk
+
+using namespace tk;
+
+extern "C" {
+
+const char* topk_status_string(int status) {
+  switch (status) {
+    case TOPK_OK: return "TOPK_OK";
+    case TOPK_EINVAL: return "TOPK_EINVAL: invalid argument";
+    case TOPK_EUNSUPPORTED: return "TOPK_EUNSUPPORTED: valid but not implemented by this build";
+    case TOPK_ECUDA: return "TOPK_ECUDA: CUDA call or kernel launch failed";
+    case TOPK_EWORKSPACE: return "TOPK_EWORKSPACE: workspace missing or too small";
+  }
+  return "unknown topk status";
+}
+
+size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int kb, int d) {
+  DeviceInfo dev;
+  if (current_device_info(&dev)) return 0;
+  Plan pl;
+  if (op == TOPK_OP_EXACT) return 0;
+  if (check_common(rows, n, k, b, kb)) return 0;
+  if (op == TOPK_OP_BUCKETED) {
+    // Size for the slower-path plan too so one workspace fits either path.
+    Plan p2;
+    if (plan_select(true, rows, n, b, kb, dev, &pl) && plan_select(false, rows, n, b, kb, dev, &pl))
+      return 0;
+    if (plan_select(false, rows, n, b, kb, dev, &p2) == TOPK_OK)
+      return std::max(pl.workspace(), p2.workspace());
+    return pl.workspace();
+  }
+  if (op == TOPK_OP_SCORE) {
+    if (kLanes % b) return 0;
+    if (plan_score(rows, n, b, kb, d, dev, &pl)) return 0;
+    return pl.workspace();
+  }
+  return 0;
+}
+
+int topk_bucketed(const float* scores, int64_t rows, int64_t n, int k, int b, int kb,
+                  float* out_vals, int32_t* out_idx, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
+  int rc = check_common(rows, n, k, b, kb);
+  if (rc) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev))) return rc;
+  const bool fast = select_fast(scores, n, b);
+  Plan pl;
+  if ((rc = plan_select(fast, rows, n, b, kb, dev, &pl))) return rc;
+  if (plan_needs_workspace(pl, rows, n)) {
+    if (!workspace || workspace_bytes < pl.workspace()) return TOPK_EWORKSPACE;
+    if (!aligned16(workspace)) return TOPK_EINVAL;
+  }
+  SelectArgs a;
+  a.x = scores;
+  a.k = k;
+  a.b = b;
+  a.out_vals = out_vals;
+  a.out_idx = out_idx;
+  a.rs = make_split(pl, rows, n, workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (kb) {
+    case 1: return launch_select_kb<1>(fast, pl, a, st);
+    case 2: return launch_select_kb<2>(fast, pl, a, st);
+    case 3: return launch_select_kb<3>(fast, pl, a, st);
+    default: return launch_select_kb<4>(fast, pl, a, st);
+  }
+}
+
+int topk_exact(const float* scores, int64_t rows, int64_t n, int k, float* out_vals,
+               int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
+  if (rows < 1 || n < 1 || k < 1 || n > kMaxN) return TOPK_EINVAL;
+  if (k > kMaxK || rows > 2147483647LL) return TOPK_EUNSUPPORTED;
+  DeviceInfo dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  ExactSmem L{n <= kSortCap ? host_next_pow2(static_cast<int>(n)) : 0,
+              host_next_pow2(k)};
+  const size_t smem = L.total();
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  if ((rc = prepare_kernel(exact_topk_kernel))) return rc;
+  clear_launch_error();
+  exact_topk_kernel<<<static_cast<unsigned>(rows), kExactThreads, smem,
+                      static_cast<cudaStream_t>(stream)>>>(scores, n, k, L.sel_cap, out_vals,
+                                                           out_idx);
+  return launch_status();
+}
+
+int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,
+               int64_t k_batch_stride, int k, int b, int kb, float* out_vals, int32_t* out_idx,
+               float* out_scores, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !K || !out_vals || !out_idx) return TOPK_EINVAL;
+  int rc = check_common(rows, n, k, b, kb);
+  if (rc) return rc;
+  if (k_batch_stride < 0) return TOPK_EINVAL;
+  if (d != 128 && d != 256) return TOPK_EUNSUPPORTED;
+  if (kLanes % b) return TOPK_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(K) || (k_batch_stride % 8) != 0) return TOPK_EINVAL;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev))) return rc;
+  Plan pl;
+  if ((rc = plan_score(rows, n, b, kb, d, dev, &pl))) return rc;
+  if (plan_needs_workspace(pl, rows, n)) {
+    if (!workspace || workspace_bytes < pl.workspace()) return TOPK_EWORKSPACE;
+    if (!aligned16(workspace)) return TOPK_EINVAL;
+  }
+  ScoreArgs a;
+  a.q = q;
+  a.K = K;
+  a.kstride = k_batch_stride;
+  a.k = k;
+  a.b = b;
+  a.out_vals = out_vals;
+  a.out_idx = out_idx;
+  a.out_scores = out_scores;
+  a.rs = make_split(pl, rows, n, workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (kb) {
+    case 1: return launch_score_k<1>(d, pl, a, st);
+    case 2: return launch_score_k<2>(d, pl, a, st);
+    case 3: return launch_score_k<3>(d, pl, a, st);
+    default: return launch_score_k<4>(d, pl, a, st);
+  }
+}
+
+int topk_device_status(int* status_out) {
+  if (!status_out) return TOPK_EINVAL;
+  if (cudaDeviceSynchronize() != cudaSuccess) return TOPK_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return TOPK_ECUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return TOPK_ECUDA;
+  *status_out = v;
+  return TOPK_OK;
+}
+
+}  // extern "C"

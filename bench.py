@@ -1,0 +1,455 @@
+"""Benchmark: bucketed approximate top-k on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config decode|tiny|vocab|link|long-b128-kb1 ...]
+
+One step is one pass of the whole hot path over one batch of resident input.
+The default workload is the sparse-attention decode selection: 16 x 32 rows,
+each a bf16 query (d = 128) scored against its own 32768 x 128 bf16 key matrix
+(4 GiB of keys in total, larger than L2), then bucketed top-k with k = 512,
+b = 256, k_b = 2 -- one fused kernel launch per step.
+
+The metric is "bucketed top-k GB/s of scores read": the bytes of score input the
+step must read (the key matrices and queries for the fused step), plus the
+output, divided by the step's device time.  rows/s and the recall against exact
+top-k (with Eq. (1) of "Approximate Top-k for Increased Parallelism" beside it)
+ride along.  Timing protocol after that paper's benchmark appendix: warm-up
+launches, then device-side CUDA events around K steps.
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+inputs (rows are independent; no collective on the data path); the time is the
+maximum over ranks and `value` counts the bytes of all ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "bucketed top-k GB/s of scores read vs HBM peak; rows/s; recall@k vs Eq.(1)"
+
+# name -> workload description.  kind: "score" (fused q.K + selection) or "select".
+CONFIGS = {
+    "tiny": dict(kind="select", rows=8, n=4096, k=64, b=128, kb=1, dist="normal"),
+    "decode": dict(kind="score", batch=16, heads=32, n=32768, d=128, k=512, b=256, kb=2),
+    "vocab": dict(kind="select", rows=256, n=131072, k=50, b=512, kb=1, dist="vocab"),
+    "link": dict(kind="score", queries=1024, n=1 << 20, d=256, k=100, b=1024, kb=1),
+    # a quarter of the decode rows (1 GiB of keys): the case profiled with ncu --set full
+    "decode-quarter": dict(kind="score", batch=4, heads=32, n=32768, d=128, k=512, b=256, kb=2),
+}
+for _b in (128, 256, 512):
+    for _kb in (1, 2, 4):
+        CONFIGS["long-b%d-kb%d" % (_b, _kb)] = dict(kind="select", rows=256, n=131072, k=512,
+                                                    b=_b, kb=_kb, dist="uniform")
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.15)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workloads
+class Workload:
+    """Resident device inputs for one config, plus the step function."""
+
+    def __init__(self, name: str, device, seed_offset: int = 0):
+        from approximate_top_selection_b200 import inputs
+
+        self.name, self.cfg, self.device = name, CONFIGS[name], device
+        c = self.cfg
+        seed = inputs.SEEDS[name.split("-")[0]] + seed_offset
+        if c["kind"] == "score":
+            if "batch" in c:
+                self.rows = c["batch"] * c["heads"]
+                self.q, self.K = inputs.decode_inputs(c["batch"], c["heads"], c["n"], c["d"], seed,
+                                                      device=device)
+            else:
+                self.rows = c["queries"]
+                self.q, self.K = inputs.link_inputs(c["queries"], c["n"], c["d"], seed,
+                                                    device=device)
+            self.in_bytes = self.q.numel() * 2 + self.K.numel() * 2
+        else:
+            self.rows = c["rows"]
+            if c["dist"] == "normal":
+                self.x = inputs.normal_rows(c["rows"], c["n"], seed, device=device)
+            elif c["dist"] == "vocab":
+                self.x = inputs.vocab_logits(c["rows"], c["n"], seed, device=device)
+            else:
+                self.x = inputs.uniform_rows(c["rows"], c["n"], seed, device=device)
+            self.in_bytes = self.x.numel() * 4
+        self.out_bytes = self.rows * c["k"] * 8
+        self.bytes = self.in_bytes + self.out_bytes
+        self.larger_than_l2 = self.in_bytes > 126 * 2 ** 20
+
+    def step(self, stream=None):
+        import approximate_top_selection_b200 as atk
+
+        c = self.cfg
+        if c["kind"] == "score":
+            return atk.score_topk(self.q, self.K, c["k"], c["b"], c["kb"], stream=stream)
+        return atk.topk_bucketed(self.x, c["k"], c["b"], c["kb"], stream=stream)
+
+    def describe(self):
+        c = dict(self.cfg)
+        c["workload"] = self.name
+        return c
+
+
+def _kernel_name(cfg) -> str:
+    if cfg["kind"] == "score":
+        return "score_select_gemv"
+    return "bucket_select_tma"
+
+
+def _rotations(w: Workload) -> int:
+    """Input copies needed so that consecutive steps do not hit in L2."""
+    return 1 if w.larger_than_l2 else max(2, math.ceil(3 * 126 * 2 ** 20 / w.in_bytes))
+
+
+def recall_report(w: Workload):
+    """Recall of the step's selection against exact top-k on the same scores."""
+    import approximate_top_selection_b200 as atk
+    from oracle import recall as rc
+
+    c = w.cfg
+    if c["kind"] == "score":
+        rows = min(w.rows, 64)
+        _, bi, s = atk.score_topk(w.q[:rows], w.K[:rows] if w.K.dim() == 3 else w.K, c["k"],
+                                  c["b"], c["kb"], return_scores=True)
+    else:
+        rows = min(w.rows, 256)
+        s = w.x[:rows]
+        _, bi = atk.topk_bucketed(s, c["k"], c["b"], c["kb"])
+    _, ei = atk.topk_exact(s, c["k"])
+    r = rc.recall(bi.cpu().numpy(), ei.cpu().numpy())
+    n = c["n"]
+    out = {"mean": float(r.mean()), "rows": rows, "eq1": rc.eq1_expected_recall(c["k"], c["b"], c["kb"])}
+    if n % c["b"] == 0 and c["kind"] == "score" or c.get("dist") == "uniform":
+        out["exact_expectation_iid"] = rc.expected_recall_exact(n, c["k"], c["b"], c["kb"])
+    return out
+
+
+def cpu_baseline(w: Workload, budget_s: float = 10.0):
+    """The oracle, as it stands, on the host cores over a bounded row sample."""
+    import oracle
+
+    oracle.build()
+    threads = oracle.max_threads()
+    oracle.set_threads(threads)
+    c = w.cfg
+
+    def run(rows):
+        t0 = time.perf_counter()
+        if c["kind"] == "score":
+            q = w.q[:rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+            K = (w.K[:rows] if w.K.dim() == 3 else w.K).cpu().contiguous().view(torch.int16)
+            K = K.numpy().view(np.uint16)
+            t0 = time.perf_counter()
+            oracle.score_topk(q, K, c["k"], c["b"], c["kb"])
+        else:
+            x = w.x[:rows].cpu().numpy()
+            t0 = time.perf_counter()
+            oracle.bucketed(x, c["k"], c["b"], c["kb"])
+        return time.perf_counter() - t0
+
+    probe = min(w.rows, max(1, threads))
+    t = run(probe)
+    rows = int(min(w.rows, max(probe, probe * budget_s / max(t, 1e-6))))
+    if rows > probe:
+        t = run(rows)
+    else:
+        rows = probe
+    per_row = w.bytes / w.rows
+    return {"value": rows * per_row / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "%d of %d rows of the %s workload (%.1f s)" % (rows, w.rows, w.name, t),
+            "rows_per_s": rows / t}
+
+
+# ---------------------------------------------------------------- runs
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def run_ours(args, world, rank, local):
+    import approximate_top_selection_b200 as atk
+
+    atk.load_library()
+    dev = torch.device("cuda", local)
+    w = Workload(args.config, dev, seed_offset=rank)
+    nrot = _rotations(w)
+    extra = [Workload(args.config, dev, seed_offset=rank + 101 * (j + 1)) for j in range(nrot - 1)]
+    works = [w] + extra
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        works[i % nrot].step()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        ev0.record(stream)
+        for i in range(args.steps):
+            works[i % nrot].step()
+        ev1.record(stream)
+        barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    hbm, _, peak_src = _peaks()
+    achieved = w.bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": achieved * world,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16->f32" if w.cfg["kind"] == "score" else "f32",
+        "data": "synthetic (seeded; shapes of the pages' workloads)",
+        "config": dict(w.describe(), l2="inputs larger than L2" if nrot == 1 else
+                       "%d rotating input copies (%.0f MiB) defeat L2" %
+                       (nrot, nrot * w.in_bytes / 2 ** 20)),
+        "rows_per_s": w.rows * world / (ms_step * 1e-3),
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": _kernel_name(w.cfg), "peak_source": peak_src + " hbm_gbs"},
+        "clocks": clk.summary(),
+    }
+    if not args.no_recall:
+        line["recall"] = recall_report(w)
+    if not args.no_e2e:
+        line["e2e"] = e2e(w, args, world)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
+    return line
+
+
+def e2e(w: Workload, args, world):
+    """Same metric through the public API with host buffers: per step, pinned
+    host -> device copy of the inputs, the call, device -> host of the result."""
+    import approximate_top_selection_b200 as atk
+
+    c = w.cfg
+    steps = max(1, min(args.steps, args.e2e_steps))
+    if c["kind"] == "score":
+        hq = torch.empty(w.q.shape, dtype=w.q.dtype, pin_memory=True)
+        hK = torch.empty(w.K.shape, dtype=w.K.dtype, pin_memory=True)
+        hq.copy_(w.q)
+        hK.copy_(w.K)
+        dq, dK = torch.empty_like(w.q), torch.empty_like(w.K)
+        h2d = hq.numel() * 2 + hK.numel() * 2
+    else:
+        hx = torch.empty(w.x.shape, dtype=w.x.dtype, pin_memory=True)
+        hx.copy_(w.x)
+        dx = torch.empty_like(w.x)
+        h2d = hx.numel() * 4
+    hv = torch.empty(w.rows, c["k"], dtype=torch.float32, pin_memory=True)
+    hi = torch.empty(w.rows, c["k"], dtype=torch.int32, pin_memory=True)
+    stream = torch.cuda.current_stream()
+
+    def one():
+        if c["kind"] == "score":
+            dq.copy_(hq, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            v, i = atk.score_topk(dq, dK, c["k"], c["b"], c["kb"])
+        else:
+            dx.copy_(hx, non_blocking=True)
+            v, i = atk.topk_bucketed(dx, c["k"], c["b"], c["kb"])
+        hv.copy_(v, non_blocking=True)
+        hi.copy_(i, non_blocking=True)
+
+    one()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        one()
+    ev1.record(stream)
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world) / steps
+    return {"value": w.bytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": w.rows * c["k"] * 8,
+            "ms_per_step": ms, "steps": steps}
+
+
+def run_reference(args, world, rank, local):
+    """The oracle on the host cores: each step is a bounded row sample."""
+    import oracle
+
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    w = Workload(args.config, dev)
+    oracle.build()
+    threads = oracle.max_threads()
+    oracle.set_threads(threads)
+    c = w.cfg
+    # sample size: about 1 s of oracle work per step
+    probe = cpu_baseline(w, budget_s=1.0)
+    rows = max(1, min(w.rows, int(probe["rows_per_s"] * 1.0)))
+    if c["kind"] == "score":
+        q = w.q[:rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        K = (w.K[:rows] if w.K.dim() == 3 else w.K).cpu().contiguous().view(torch.int16)
+        K = K.numpy().view(np.uint16)
+        step = lambda: oracle.score_topk(q, K, c["k"], c["b"], c["kb"])  # noqa: E731
+    else:
+        x = w.x[:rows].cpu().numpy()
+        step = lambda: oracle.bucketed(x, c["k"], c["b"], c["kb"])  # noqa: E731
+    for _ in range(min(args.warmup, 3)):
+        step()
+    steps = max(1, min(args.steps, 20))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / steps
+    per_row = w.bytes / w.rows
+    value = rows * per_row / dt / 1e9
+    sample = "%d of %d rows of the %s workload per step" % (rows, w.rows, w.name)
+    return {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": min(args.warmup, 3), "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate / f32 select",
+            "data": "synthetic", "impl": "reference", "config": w.describe(),
+            "rows_per_s": rows / dt,
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=16)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-recall", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        line = run_reference(args, world, rank, int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(line))
+        return
+    world, rank, local = setup_dist(args)
+    line = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

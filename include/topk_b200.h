@@ -1,0 +1,119 @@
+/*
+ * topk_b200.h -- C ABI of the B200 (sm_100a) bucketed approximate top-k library.
+ *
+ * Method: "Approximate Top-k for Increased Parallelism" (Key, Ribar, Cattaneo,
+ * Hudlass-Galley, Orr; arXiv 2412.04358), pith.science review page, section
+ * "What carries the argument" and Fig. 2: a row of n scores is split into b
+ * interleaved buckets (element i goes to bucket i mod b, "The reading"), an
+ * exact top-k_b is kept per bucket (Stage 1), and when the b*k_b candidates
+ * exceed k a final exact top-k keeps the k best (Stage 2).
+ *
+ * Common conventions
+ *   - Every pointer argument named *_dev is CUDA device memory owned by the
+ *     caller; the library keeps no pointer after the call returns.
+ *   - Matrices are row-major and contiguous: row r of an [rows x n] array
+ *     starts at element r*n.
+ *   - Total order: a larger value ranks first; equal values (IEEE equality, so
+ *     -0.0 ties +0.0) rank by lower index; NaN ranks above +inf and all NaNs
+ *     are equal.
+ *   - Outputs out_vals[rows*k] / out_idx[rows*k] hold, per row, the selected
+ *     elements best-first.  When fewer than k elements are selected (fewer
+ *     candidates than k, or n < k), the remaining slots hold -inf and -1.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  Argument errors are detected on the host before any
+ *     work is queued; nothing throws across the ABI.
+ *   - The workspace (when required) is caller-owned device memory of at least
+ *     topk_workspace_bytes(...) bytes that MUST be zero-filled before its first
+ *     use.  Every call leaves it zero-filled again when it completes on the GPU,
+ *     so one workspace can be reused for any later call.  Calls that overlap on
+ *     the GPU (different streams) must not share a workspace.
+ *   - Device-side waits are bounded in time; a wait that expires records a
+ *     code readable with topk_device_status() and the kernel returns early.
+ */
+#ifndef TOPK_B200_H
+#define TOPK_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TOPK_OK = 0,          /* queued successfully */
+    TOPK_EINVAL = 1,      /* bad argument: null pointer, size < 1, k_b outside [1,4], n >= 2^31 */
+    TOPK_EUNSUPPORTED = 2,/* valid but outside what this build implements (see each call) */
+    TOPK_ECUDA = 3,       /* a CUDA call or kernel launch failed */
+    TOPK_EWORKSPACE = 4   /* workspace missing or smaller than topk_workspace_bytes() */
+} topk_status;
+
+typedef enum {
+    TOPK_OP_BUCKETED = 0,
+    TOPK_OP_EXACT = 1,
+    TOPK_OP_SCORE = 2
+} topk_op;
+
+/* Bytes of workspace a call of `op` with these sizes needs on the current
+ * device (0 when none).  Unused arguments are ignored (d for BUCKETED/EXACT,
+ * b and kb for EXACT).  Returns 0 as well for invalid sizes. */
+size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int kb, int d);
+
+/* Two-stage bucketed approximate top-k ("What carries the argument"; Fig. 2).
+ *   scores_dev  [rows x n] float32 scores.
+ *   k           number of outputs per row, 1 <= k <= 16384.
+ *   b           number of interleaved buckets, 1 <= b <= 1024.
+ *   kb          candidates kept per bucket, 1 <= kb <= 4 (register queues).
+ *   out_vals_dev[rows x k] float32: the selected scores (input bits unchanged).
+ *   out_idx_dev [rows x k] int32: their column indices.
+ * The result equals the CPU definition bit for bit.  Fast path: n % 4 == 0,
+ * scores 16-byte aligned and b dividing 1024; other shapes take a slower
+ * general path.  Returns TOPK_EUNSUPPORTED for b > 1024 or k > 16384. */
+int topk_bucketed(const float *scores_dev, int64_t rows, int64_t n, int k, int b, int kb,
+                  float *out_vals_dev, int32_t *out_idx_dev, void *workspace_dev,
+                  size_t workspace_bytes, void *stream);
+
+/* Exact top-k of every row under the total order above: the baseline the
+ * page compares against (Fig. 1, "exact top-k implementations") and the
+ * Stage-2 primitive.  1 <= k <= 16384 (else TOPK_EUNSUPPORTED).  No workspace:
+ * pass NULL / 0. */
+int topk_exact(const float *scores_dev, int64_t rows, int64_t n, int k, float *out_vals_dev,
+               int32_t *out_idx_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
+
+/* Fused selector: score[r][i] = sum_t q[r][t] * K_r[i][t] (bf16 inputs, fp32
+ * accumulation; no 1/sqrt(d) scaling), then topk_bucketed on each row of
+ * scores -- the sparse-attention selector that scores the current query
+ * against the whole key cache before a global top-K ("Recall Before You Rank"
+ * abstract; STARC page, Fig. 3: q in R^{1 x d_h}, K in R^{L x d_h}).  The
+ * score matrix is not materialised.
+ *   q_dev        [rows x d] bf16 (raw 16-bit patterns), 16-byte aligned.
+ *   K_dev        bf16 keys; row r uses K_r = K_dev + r*k_batch_stride
+ *                elements, an [n x d] row-major matrix.  k_batch_stride = 0
+ *                shares one key matrix between all rows.  16-byte aligned.
+ *   d            128 or 256 (else TOPK_EUNSUPPORTED).
+ *   k, b, kb     as in topk_bucketed, with b dividing 1024 (else
+ *                TOPK_EUNSUPPORTED).
+ *   out_scores_dev  nullable [rows x n] float32: when given, receives the
+ *                fp32 scores the selection ran on (for checking).
+ * Output values are the fp32 scores (a zero score is returned as +0.0 and a
+ * NaN score as the quiet NaN 0x7FFFFFFF). */
+int score_topk(const uint16_t *q_dev, int64_t rows, int d, const uint16_t *K_dev, int64_t n,
+               int64_t k_batch_stride, int k, int b, int kb, float *out_vals_dev,
+               int32_t *out_idx_dev, float *out_scores_dev, void *workspace_dev,
+               size_t workspace_bytes, void *stream);
+
+/* Human-readable name of a topk_status value (static string). */
+const char *topk_status_string(int status);
+
+/* Reads and clears the device-side status word of the current device: 0 when
+ * no bounded wait has expired since the last read, else a bit set of
+ * TOPK_DEV_* codes.  Synchronises the device. */
+int topk_device_status(int *status_out);
+
+#define TOPK_DEV_WAIT_TIMEOUT 1 /* a bulk-copy wait in a streaming kernel expired */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOPK_B200_H */

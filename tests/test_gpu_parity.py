@@ -1,0 +1,277 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Selection (topk_bucketed, topk_exact) must match bit for bit: values and
+indices.  Fused scoring (score_topk) must agree with the oracle's fp64 scores
+within 2e-3 relative (floor 2^-10 * |q| |K_i|), the selection the GPU made on
+its own fp32 scores must equal the oracle's selection on those same scores bit
+for bit, and the index sets must match except where the oracle's decision is
+fragile (a bucket's k_b-th/(k_b+1)-th gap or the k-th/(k+1)-th candidate gap
+below the tolerance).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import approximate_top_selection_b200 as atk
+from approximate_top_selection_b200 import inputs
+from oracle import recall as rc
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu(oracle_mod):
+    if not torch.cuda.is_available():
+        pytest.fail("these tests need a CUDA device")
+    atk.load_library()
+    yield
+    assert atk.topk_device_status() == 0
+
+
+def same_bits(a, b) -> bool:
+    a = np.ascontiguousarray(np.asarray(a, np.float32))
+    b = np.ascontiguousarray(np.asarray(b, np.float32))
+    return a.shape == b.shape and np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def check_bucketed(x_cpu: torch.Tensor, k, b, kb, oracle_mod, x_dev=None, rows_subset=None):
+    x_dev = x_cpu.to(DEV) if x_dev is None else x_dev
+    v, i = atk.topk_bucketed(x_dev, k, b, kb)
+    torch.cuda.synchronize()
+    v, i = v.cpu().numpy(), i.cpu().numpy()
+    xs = x_cpu.numpy() if rows_subset is None else x_cpu.numpy()[rows_subset]
+    ov, oi = oracle_mod.bucketed(xs, k, b, kb)
+    if rows_subset is not None:
+        v, i = v[rows_subset], i[rows_subset]
+    bad = np.nonzero(~np.all(oi == i, axis=1))[0]
+    assert bad.size == 0, "index mismatch in rows %s (k=%d b=%d kb=%d)" % (bad[:5], k, b, kb)
+    assert same_bits(v, ov), "value bits differ"
+    return v, i
+
+
+# ------------------------------------------------------------------ bucketed
+def test_tiny_config(oracle_mod):
+    """8 rows x 4096 N(0,1), k=64, b=128, k_b=1 (final exact top-64 of 128)."""
+    x = inputs.normal_rows(8, 4096, inputs.SEEDS["tiny"])
+    check_bucketed(x, 64, 128, 1, oracle_mod)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_shapes(oracle_mod, seed):
+    """Random small shapes: ragged tails, b > n, k > C (padding), every k_b,
+    fast (b | 1024, n % 4 == 0) and general paths."""
+    rng = np.random.default_rng(100 + seed)
+    for t in range(12):
+        rows = int(rng.integers(1, 6))
+        n = int(rng.integers(1, 9000))
+        b = int(rng.choice([1, 2, 3, 8, 32, 100, 128, 256, 512, 1000, 1024]))
+        kb = int(rng.integers(1, 5))
+        k = int(rng.integers(1, 700))
+        kind = t % 3
+        if kind == 0:
+            x = inputs.normal_rows(rows, n, seed * 100 + t)
+        elif kind == 1:
+            x = inputs.integer_rows(rows, n, 5, seed * 100 + t)
+        else:
+            x = inputs.special_rows(rows, n, seed * 100 + t)
+        check_bucketed(x, k, b, kb, oracle_mod)
+
+
+def test_special_values_fast_path(oracle_mod):
+    """NaN, +-inf, +-0 and ties through the TMA path (n % 4 == 0, b | 1024)."""
+    x = inputs.special_rows(16, 8192, 7)
+    for (k, b, kb) in [(64, 128, 1), (100, 32, 4), (512, 256, 2), (30, 1, 4), (9, 1024, 3)]:
+        check_bucketed(x, k, b, kb, oracle_mod)
+
+
+def test_misaligned_rows_take_general_path(oracle_mod):
+    """A base pointer that is not 16-byte aligned, and n % 4 != 0."""
+    big = inputs.normal_rows(1, 4 * 3001 + 1, 9).reshape(-1)
+    x = big[1:].reshape(4, 3001)
+    xd = big.to(DEV)[1:].reshape(4, 3001)
+    check_bucketed(x.contiguous(), 50, 64, 2, oracle_mod, x_dev=xd)
+
+
+def test_split_rows_are_merged(oracle_mod):
+    """Few long rows: each row is streamed by several CTAs and merged by the
+    last one to finish (ticket in the workspace)."""
+    x = inputs.normal_rows(3, 400000, 11)
+    check_bucketed(x, 100, 512, 2, oracle_mod)
+    x = inputs.integer_rows(2, 1 << 20, 50, 12)  # ties everywhere
+    check_bucketed(x, 300, 256, 4, oracle_mod)
+    x = inputs.normal_rows(1, 999999, 13)  # general path, split
+    check_bucketed(x, 64, 100, 3, oracle_mod)
+
+
+def test_many_rows_per_cta(oracle_mod):
+    """More rows than resident CTAs: CTA ranges hold several rows and cut rows."""
+    x = inputs.uniform_rows(3000, 2048, 14)
+    check_bucketed(x, 16, 64, 1, oracle_mod)
+    x = inputs.uniform_rows(2500, 1001, 15)
+    check_bucketed(x, 20, 50, 2, oracle_mod)
+
+
+def test_workspace_reuse_across_shapes(oracle_mod):
+    """One workspace, calls of different shapes back to back: the tickets the
+    merge uses are left at zero by every call."""
+    nbytes = max(atk.topk_workspace_bytes(atk.TOPK_OP_BUCKETED, r, n, k, b, kb)
+                 for (r, n, k, b, kb) in [(2, 300000, 50, 256, 2), (5, 100000, 64, 128, 1)])
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
+    for it in range(3):
+        for (r, n, k, b, kb) in [(2, 300000, 50, 256, 2), (5, 100000, 64, 128, 1)]:
+            x = inputs.normal_rows(r, n, 1000 * it + r)
+            v, i = atk.topk_bucketed(x.to(DEV), k, b, kb, workspace=ws)
+            ov, oi = oracle_mod.bucketed(x.numpy(), k, b, kb)
+            assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+    torch.cuda.synchronize()
+    assert int(ws.count_nonzero()) <= nbytes  # slots may hold data; tickets must be zero
+    tick = ws[:256].view(torch.int32)
+    assert int(tick.abs().sum()) == 0
+
+
+def test_vocab_config_full(oracle_mod):
+    """256 rows x 131072 logits (N(0,1) + Zipf(1.1) rank offset), k=50, b=512, k_b=1."""
+    x = inputs.vocab_logits(256, 131072, inputs.SEEDS["vocab"])
+    check_bucketed(x, 50, 512, 1, oracle_mod)
+
+
+@pytest.mark.parametrize("b", [128, 256, 512])
+@pytest.mark.parametrize("kb", [1, 2, 4])
+def test_long_context_sweep(oracle_mod, b, kb):
+    """256 rows x 131072 iid U(0,1), k=512 (parity on a row sample), plus
+    adversarial rows whose top-k sit in as few residue classes as possible:
+    recall equals the worst case of Eq. (2) exactly."""
+    seed = inputs.SEEDS["long"] + 16 * b + kb
+    x = inputs.uniform_rows(256, 131072, seed)
+    sample = np.arange(0, 256, 16)
+    check_bucketed(x, 512, b, kb, oracle_mod, rows_subset=sample)
+    adv = inputs.adversarial_rows(8, 131072, 512, b, seed + 1)
+    _, gi = check_bucketed(adv, 512, b, kb, oracle_mod)
+    _, ei = oracle_mod.exact(adv.numpy(), 512)
+    r = rc.recall(gi, ei)
+    assert np.all(np.abs(r - rc.eq2_worst_recall(131072, 512, b, kb)) < 1e-12)
+
+
+@pytest.mark.parametrize("n,k,b,kb", [(4096, 64, 128, 1), (32768, 512, 256, 2),
+                                      (8192, 256, 64, 4)])
+def test_recall_band_on_gpu(oracle_mod, n, k, b, kb):
+    """Recall of the GPU result over 10^4 iid uniform rows (2000 for the larger
+    shapes): within 3 SE of the exact finite-n expectation, and not more than
+    3 SE below Eq. (1)."""
+    rows = 10000 if n <= 4096 else 2000
+    x = inputs.uniform_rows(rows, n, 77 + n + kb).to(DEV)
+    _, bi = atk.topk_bucketed(x, k, b, kb)
+    _, ei = atk.topk_exact(x, k)
+    bi, ei = bi.cpu().numpy(), ei.cpu().numpy()
+    # the exact reference itself is checked against the oracle on a sample
+    _, oi = oracle_mod.exact(x[:64].cpu().numpy(), k)
+    assert np.array_equal(ei[:64], oi)
+    r = rc.recall(bi, ei)
+    mean, se = r.mean(), r.std(ddof=1) / math.sqrt(rows)
+    assert abs(mean - rc.expected_recall_exact(n, k, b, kb)) <= 3 * se
+    assert mean >= rc.eq1_expected_recall(k, b, kb) - 3 * se
+
+
+# ------------------------------------------------------------------ exact
+@pytest.mark.parametrize("rows,n,k", [(8, 4096, 64), (4, 1000, 1000), (3, 77, 200),
+                                      (16, 8192, 512), (4, 8193, 50), (64, 131072, 50),
+                                      (2, 131072, 16384), (5, 16000, 16000), (2, 20000, 16384),
+                                      (3, 300001, 999)])
+def test_exact_matches_oracle(oracle_mod, rows, n, k):
+    x = inputs.normal_rows(rows, n, rows * 7 + n + k)
+    v, i = atk.topk_exact(x.to(DEV), k)
+    ov, oi = oracle_mod.exact(x.numpy(), k)
+    assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+
+
+def test_exact_ties_and_specials(oracle_mod):
+    for (rows, n, k, levels) in [(4, 50000, 3000, 3), (2, 100000, 77, 1), (3, 40000, 5000, 2)]:
+        x = inputs.integer_rows(rows, n, levels, n + k)
+        v, i = atk.topk_exact(x.to(DEV), k)
+        ov, oi = oracle_mod.exact(x.numpy(), k)
+        assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+    x = inputs.special_rows(4, 30000, 5)
+    v, i = atk.topk_exact(x.to(DEV), 700)
+    ov, oi = oracle_mod.exact(x.numpy(), 700)
+    assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+
+
+# ------------------------------------------------------------------ scoring
+def _bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def check_scores(q: torch.Tensor, K: torch.Tensor, k, b, kb, oracle_mod, rows_subset=None):
+    """q, K on the device.  Returns the GPU outputs after all checks."""
+    v, i, s = atk.score_topk(q, K, k, b, kb, return_scores=True)
+    torch.cuda.synchronize()
+    v, i, s = v.cpu().numpy(), i.cpu().numpy(), s.cpu().numpy()
+    rows = q.shape[0]
+    sub = np.arange(rows) if rows_subset is None else np.asarray(rows_subset)
+    # (1) the selection on the GPU's own scores is the oracle's, bit for bit
+    ov, oi = oracle_mod.bucketed(s[sub], k, b, kb)
+    assert np.array_equal(i[sub], oi) and same_bits(v[sub], ov)
+    # (2) scores within tolerance of the fp64 oracle
+    tsub = torch.as_tensor(sub, device=q.device)
+    qs = q[tsub]
+    Ks = K[tsub] if K.dim() == 3 else K
+    ref = oracle_mod.scores(_bits(qs), _bits(Ks))
+    qn = torch.linalg.vector_norm(qs.float().cpu(), dim=1).double().numpy()
+    kn = torch.linalg.vector_norm(Ks.float().cpu(), dim=-1).double().numpy()
+    scale = qn[:, None] * (kn if kn.ndim == 2 else kn[None, :])
+    tol = 2e-3 * np.maximum(np.abs(ref), 2.0 ** -10 * scale)
+    err = np.abs(s[sub].astype(np.float64) - ref)
+    assert np.all(err <= tol), float((err / tol).max())
+    # (3) index sets equal except at fragile decisions of the oracle: a near-tie
+    # (within twice the tolerance) at a bucket's k_b-th/(k_b+1)-th boundary or at
+    # the k-th/(k+1)-th candidate boundary, with the element inside that band.
+    rv, ri = oracle_mod.bucketed(ref, k, b, kb)
+    gi = i[sub]
+    for row in range(len(sub)):
+        a, g = set(ri[row][ri[row] >= 0].tolist()), set(gi[row][gi[row] >= 0].tolist())
+        diff = a ^ g
+        if not diff:
+            continue
+        sc = ref[row].astype(np.float64)
+        T = 2 * float(tol[row].max())
+        cols = [np.sort(sc[j::b])[::-1] for j in range(b)]
+        cand = np.sort(np.concatenate([c[:kb] for c in cols]))[::-1]
+        for idx in diff:
+            col = cols[idx % b]
+            near_bucket = (len(col) > kb and col[kb - 1] - col[kb] <= T
+                           and col[kb] - T <= sc[idx] <= col[kb - 1] + T)
+            near_stage2 = (len(cand) > k and cand[k - 1] - cand[k] <= T
+                           and cand[k] - T <= sc[idx] <= cand[k - 1] + T)
+            assert near_bucket or near_stage2, (row, idx)
+    return v, i, s
+
+
+def test_score_small_per_row_keys(oracle_mod):
+    q, K = inputs.decode_inputs(2, 3, 5000, 128, 21)
+    check_scores(q.to(DEV), K.to(DEV), 512, 256, 2, oracle_mod)
+
+
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb", [1, 4])
+def test_score_shapes(oracle_mod, d, kb):
+    q, K = inputs.decode_inputs(1, 5, 3333, d, 22 + d + kb)
+    check_scores(q.to(DEV), K.to(DEV), 100, 64, kb, oracle_mod)
+    Q, Ks = inputs.link_inputs(7, 20001, d, 23 + d + kb)
+    check_scores(Q.to(DEV), Ks.to(DEV), 100, 1024, kb, oracle_mod)
+
+
+def test_score_long_rows_split(oracle_mod):
+    q, K = inputs.decode_inputs(1, 2, 300000, 128, 24)
+    check_scores(q.to(DEV), K.to(DEV), 512, 256, 2, oracle_mod)
+
+
+def test_decode_config_full(oracle_mod):
+    """16 x 32 rows, 32768 keys of d=128: sampled rows against the oracle."""
+    q, K = inputs.decode_inputs(16, 32, 32768, 128, inputs.SEEDS["decode"], device=DEV)
+    check_scores(q, K, 512, 256, 2, oracle_mod, rows_subset=[0, 1, 100, 255, 256, 400, 511])
