@@ -9,6 +9,6 @@ The Python names mirror the C ABI in include/topk_b200.h; all work runs in the
 CUDA library libtopk_b200.so (build: `python -m approximate_top_selection_b200.build`).
 """
 from ._binding import (  # noqa: F401
-    TOPK_EINVAL, TOPK_ECUDA, TOPK_EUNSUPPORTED, TOPK_EWORKSPACE, TOPK_OK, TOPK_OP_BUCKETED,
+    TOPK_EINVAL, TOPK_ECUDA, TOPK_ESCRATCH, TOPK_EUNSUPPORTED, TOPK_EWORKSPACE, TOPK_OK, TOPK_OP_BUCKETED,
     TOPK_OP_EXACT, TOPK_OP_SCORE, TopkError, library_path, load_library, score_topk,
-    topk_bucketed, topk_device_status, topk_exact, topk_status_string, topk_workspace_bytes)
+    topk_bucketed, topk_bucketed_noalloc, topk_device_status, topk_exact, topk_status_string, topk_workspace_bytes)

@@ -15,7 +15,7 @@ import torch
 
 from . import build as _build
 
-TOPK_OK, TOPK_EINVAL, TOPK_EUNSUPPORTED, TOPK_ECUDA, TOPK_EWORKSPACE = range(5)
+TOPK_OK, TOPK_EINVAL, TOPK_EUNSUPPORTED, TOPK_ECUDA, TOPK_EWORKSPACE, TOPK_ESCRATCH = range(6)
 TOPK_OP_BUCKETED, TOPK_OP_EXACT, TOPK_OP_SCORE = range(3)
 
 _lib = None
@@ -54,6 +54,8 @@ def load_library():
             lib.topk_exact.restype = i32
             lib.score_topk.argtypes = [p, i64, i32, p, i64, i64, i32, i32, i32, p, p, p, p, sz, p]
             lib.score_topk.restype = i32
+            lib.topk_bucketed_noalloc.argtypes = [p, i64, i64, i32, i32, i32, p, p, p]
+            lib.topk_bucketed_noalloc.restype = i32
             lib.topk_status_string.argtypes = [i32]
             lib.topk_status_string.restype = ctypes.c_char_p
             lib.topk_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -148,6 +150,27 @@ def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=Non
                                out_idx.data_ptr(), ws.data_ptr() if ws is not None else None,
                                ws.numel() if ws is not None else 0, sh)
     _check(st, "topk_bucketed")
+    return out_vals, out_idx
+
+
+def topk_bucketed_noalloc(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=None,
+                          out_idx=None, stream=None):
+    """topk_bucketed without a workspace: for callers that must not allocate
+    device memory when they select (the library's built-in scratch buffer is
+    used instead; see include/topk_b200.h).  Pass preallocated out_vals /
+    out_idx to allocate nothing at all on this path.  Calls on different
+    streams that overlap on the GPU race on the shared buffer."""
+    lib = load_library()
+    _cuda(scores, "scores", torch.float32)
+    if scores.dim() != 2:
+        raise ValueError("scores must be [rows, n]")
+    rows, n = scores.shape
+    with torch.cuda.device(scores.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
+        st = lib.topk_bucketed_noalloc(scores.data_ptr(), rows, n, k, b, kb, out_vals.data_ptr(),
+                                       out_idx.data_ptr(), sh)
+    _check(st, "topk_bucketed_noalloc")
     return out_vals, out_idx
 
 

@@ -325,6 +325,35 @@ int launch_score_k(int d, const Plan& pl, const ScoreArgs& a, cudaStream_t st) {
   return launch_score_kd<KB, 256>(pl, a, st);
 }
 
+// ---------------------------------------------------------------- no-alloc scratch
+// Built-in scratch of topk_bucketed_noalloc.  In host code this name is only a
+// stand-in for the symbol: the device address is looked up per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TOPK_NOALLOC_SCRATCH_BYTES];
+
+struct ScratchAddr {
+  bool init = false;
+  void* ptr = nullptr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Device address of g_noalloc_scratch on the current device (looked up once).
+int noalloc_scratch_ptr(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TOPK_ECUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  ScratchAddr& s = g_scratch_addr[dev];
+  if (!s.init) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return TOPK_ECUDA;
+    s.ptr = p;
+    s.init = true;
+  }
+  *out = s.ptr;
+  return TOPK_OK;
+}
+
 }  // namespace
 }  // namespace tk
 
@@ -339,6 +368,9 @@ const char* topk_status_string(int status) {
     case TOPK_EUNSUPPORTED: return "TOPK_EUNSUPPORTED: valid but not implemented by this build";
     case TOPK_ECUDA: return "TOPK_ECUDA: CUDA call or kernel launch failed";
     case TOPK_EWORKSPACE: return "TOPK_EWORKSPACE: workspace missing or too small";
+    case TOPK_ESCRATCH:
+      return "TOPK_ESCRATCH: the call needs more scratch than the built-in buffer of "
+             "topk_bucketed_noalloc holds";
   }
   return "unknown topk status";
 }
@@ -389,6 +421,39 @@ int topk_bucketed(const float* scores, int64_t rows, int64_t n, int k, int b, in
   a.out_idx = out_idx;
   a.rs = make_split(pl, rows, n, workspace);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (kb) {
+    case 1: return launch_select_kb<1>(fast, pl, a, st);
+    case 2: return launch_select_kb<2>(fast, pl, a, st);
+    case 3: return launch_select_kb<3>(fast, pl, a, st);
+    default: return launch_select_kb<4>(fast, pl, a, st);
+  }
+}
+
+int topk_bucketed_noalloc(const float* scores, int64_t rows, int64_t n, int k, int b, int kb,
+                          float* out_vals, int32_t* out_idx, void* stream) {
+  if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
+  int rc = check_common(rows, n, k, b, kb);
+  if (rc) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev))) return rc;
+  const bool fast = select_fast(scores, n, b);
+  Plan pl;
+  if ((rc = plan_select(fast, rows, n, b, kb, dev, &pl))) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch_ptr(&scratch))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (plan_needs_workspace(pl, rows, n)) {
+    if (pl.workspace() > static_cast<size_t>(TOPK_NOALLOC_SCRATCH_BYTES)) return TOPK_ESCRATCH;
+    // The tickets must start at zero whatever an earlier call left behind.
+    if (cudaMemsetAsync(scratch, 0, pl.ws_tickets, st) != cudaSuccess) return TOPK_ECUDA;
+  }
+  SelectArgs a;
+  a.x = scores;
+  a.k = k;
+  a.b = b;
+  a.out_vals = out_vals;
+  a.out_idx = out_idx;
+  a.rs = make_split(pl, rows, n, scratch);
   switch (kb) {
     case 1: return launch_select_kb<1>(fast, pl, a, st);
     case 2: return launch_select_kb<2>(fast, pl, a, st);

@@ -45,7 +45,9 @@ typedef enum {
     TOPK_EINVAL = 1,      /* bad argument: null pointer, size < 1, k_b outside [1,4], n >= 2^31 */
     TOPK_EUNSUPPORTED = 2,/* valid but outside what this build implements (see each call) */
     TOPK_ECUDA = 3,       /* a CUDA call or kernel launch failed */
-    TOPK_EWORKSPACE = 4   /* workspace missing or smaller than topk_workspace_bytes() */
+    TOPK_EWORKSPACE = 4,  /* workspace missing or smaller than topk_workspace_bytes() */
+    TOPK_ESCRATCH = 5     /* topk_bucketed_noalloc: the call needs more scratch than the
+                             library's built-in buffer holds (TOPK_NOALLOC_SCRATCH_BYTES) */
 } topk_status;
 
 typedef enum {
@@ -101,6 +103,35 @@ int score_topk(const uint16_t *q_dev, int64_t rows, int d, const uint16_t *K_dev
                int64_t k_batch_stride, int k, int b, int kb, float *out_vals_dev,
                int32_t *out_idx_dev, float *out_scores_dev, void *workspace_dev,
                size_t workspace_bytes, void *stream);
+
+/* Allocation-free form of topk_bucketed.  The paper has no counterpart: this
+ * entry point exists for callers that must not allocate device memory at call
+ * time -- for example a serving loop in which a cudaMalloc could synchronise
+ * the device and stall every other stream, a host framework whose memory
+ * accounting forbids allocations it did not make itself, or a plugin that may
+ * only allocate while it is being set up.  Such callers pass inputs and
+ * outputs as for topk_bucketed, but no workspace: the scratch memory the
+ * kernel needs for rows split across CTAs lives in one static device buffer
+ * of TOPK_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.
+ *   - Nothing is allocated and no allocating routine is called: no cudaMalloc,
+ *     cudaFree or library allocator.
+ *   - The first call on a device looks up that device's address of the buffer
+ *     (with the device current); make that first call before any stream
+ *     capture begins on the device.
+ *   - A call whose scratch need exceeds the buffer returns TOPK_ESCRATCH and
+ *     queues nothing; topk_workspace_bytes(TOPK_OP_BUCKETED, ...) tells the
+ *     need in advance.
+ *   - Every call on a device shares the one buffer and it keeps the previous
+ *     call's contents; the part that must start at zero is cleared on
+ *     `stream` at the start of each call.  Calls that overlap on the GPU
+ *     (different streams, no ordering between them) race on the buffer and
+ *     give wrong results: order them, or use topk_bucketed with one workspace
+ *     per stream.
+ * Results are identical to topk_bucketed's. */
+#define TOPK_NOALLOC_SCRATCH_BYTES (32u << 20)
+int topk_bucketed_noalloc(const float *scores_dev, int64_t rows, int64_t n, int k, int b, int kb,
+                          float *out_vals_dev, int32_t *out_idx_dev, void *stream);
 
 /* Human-readable name of a topk_status value (static string). */
 const char *topk_status_string(int status);
