@@ -23,7 +23,7 @@
 
 namespace tk {
 
-constexpr int kTile = 4096;  // floats per bulk copy (16 KB)
+constexpr int kTile = 8192;  // floats per bulk copy (32 KB)
 
 struct SelectArgs {
   const float* x;
@@ -53,7 +53,7 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // bytes landed; empty barrier: every consumer warp is done with the stage);
 // the kThreads consumer threads never wait for each other inside a piece.
 template <int KB>
-__global__ void __launch_bounds__(kPipeThreads) bucket_select_tma(SelectArgs p, int stages,
+__global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs p, int stages,
                                                                   int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];
   const SelectSmem L{stages, KB, cand_cap};
@@ -129,30 +129,36 @@ __global__ void __launch_bounds__(kPipeThreads) bucket_select_tma(SelectArgs p, 
     const int64_t row0 = r * n;
     const int64_t a = g - row0;
     const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
+    const uint32_t len = static_cast<uint32_t>(pend - g);  // < 2^31
+    const uint32_t pos_thread = static_cast<uint32_t>(a) + 4u * tid;
     q.reset();
-    while (g < pend) {
-
-      const int64_t c = (pend - g) < kTile ? (pend - g) : kTile;
+    for (uint32_t done = 0; done < len;) {
+      const uint32_t c = (len - done) < static_cast<uint32_t>(kTile) ? (len - done) : kTile;
       // Warp-uniform: if any lane saw the stage complete, its bytes have landed.
       const bool ok = __any_sync(0xffffffffu,
-                                 !*abort_flag &&
-                                     mbar_wait_or_abort(full + st, ph, abort_flag));
+                                 !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
-        const float* tile = ring + static_cast<size_t>(st) * kTile;
-        const uint32_t pos0 = static_cast<uint32_t>(g - row0);
+        const float* tile = ring + static_cast<size_t>(st) * kTile + 4 * tid;
+        const uint32_t pos0 = pos_thread + done;
         constexpr int U = kTile / kLanes;
-        float4 x[U];
-        uint32_t i0[U];
-        bool valid[U];
+        if (c == static_cast<uint32_t>(kTile)) {
+          float4 x[U];
+          uint32_t base[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int off = 4 * tid + kLanes * u;
-          valid[u] = off < c;
-          x[u] = valid[u] ? *reinterpret_cast<const float4*>(tile + off)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-          i0[u] = pos0 + static_cast<uint32_t>(off);
+          for (int u = 0; u < U; ++u) {
+            x[u] = *reinterpret_cast<const float4*>(tile + kLanes * u);
+            base[u] = pos0 + static_cast<uint32_t>(kLanes * u);
+          }
+          q.template offer_tile<U>(x, base);
+        } else {
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const uint32_t off = 4u * tid + static_cast<uint32_t>(kLanes * u);
+            if (off < c)
+              q.offer4(*reinterpret_cast<const float4*>(tile + kLanes * u),
+                       pos0 + static_cast<uint32_t>(kLanes * u));
+          }
         }
-        q.template offer_rows<U>(x, i0, valid);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + st);
@@ -160,13 +166,14 @@ __global__ void __launch_bounds__(kPipeThreads) bucket_select_tma(SelectArgs p, 
         st = 0;
         ph ^= 1u;
       }
-      g += c;
+      done += c;
     }
+    g = pend;
     // Piece done: publish the queues and finish (Stage 2 or cross-CTA merge).
 #pragma unroll
     for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
     group_sync(kThreads);
-    finish_piece<KB, kGatherInput>(rs, p.b, p.k, r, a, pend - row0 - a, lanebuf, cand,
+    finish_piece<KB, kGatherInput>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
                                    p.x + row0, p.out_vals, p.out_idx, piece_flag);
     group_sync(kThreads);
   }
@@ -216,11 +223,12 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, 
           const int l = tid + kThreads * w;
           const int64_t off = base + static_cast<int64_t>(W) * u + l;
           if (l < W && off < len) {
-            const uint32_t pos = static_cast<uint32_t>(a + off);
-            if (w == 0) q.template offer<0>(v[u][0], pos);
-            if (w == 1) q.template offer<1>(v[u][1], pos);
-            if (w == 2) q.template offer<2>(v[u][2], pos);
-            if (w == 3) q.template offer<3>(v[u][3], pos);
+            // queue w stores position - w (see Queues)
+            const uint32_t base = static_cast<uint32_t>(a + off) - static_cast<uint32_t>(w);
+            if (w == 0) q.template offer<0>(v[u][0], base);
+            if (w == 1) q.template offer<1>(v[u][1], base);
+            if (w == 2) q.template offer<2>(v[u][2], base);
+            if (w == 3) q.template offer<3>(v[u][3], base);
           }
         }
       }

@@ -44,6 +44,13 @@ __device__ __forceinline__ uint64_t pack(uint32_t key, uint32_t idx) {
 __device__ __forceinline__ uint32_t packed_key(uint64_t p) { return static_cast<uint32_t>(p >> 32); }
 __device__ __forceinline__ uint32_t packed_idx(uint64_t p) { return ~static_cast<uint32_t>(p); }
 
+// min that returns NaN when either operand is NaN (PTX min.NaN, sm_80+).
+__device__ __forceinline__ float fmin_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // ---------------------------------------------------------------- mbarrier / bulk copy
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

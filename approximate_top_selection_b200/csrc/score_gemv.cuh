@@ -60,7 +60,7 @@ constexpr int kScoreConsumerWarps = kThreads / 32;
 constexpr int kScorePipeThreads = kThreads + 32;
 
 template <int KB, int D>
-__global__ void __launch_bounds__(kScorePipeThreads)
+__global__ void __launch_bounds__(kScorePipeThreads, 2)
     score_select_gemv(ScoreArgs p, int stages, int cand_cap) {
   constexpr int TPK = D / 32;            // threads per key
   constexpr int KR = kThreads / TPK;     // keys per tile
@@ -202,13 +202,10 @@ __global__ void __launch_bounds__(kScorePipeThreads)
         if (off < valid) {
           const float4 v = *reinterpret_cast<const float4*>(sbuf + (blk & 1) * kLanes + off);
           const uint32_t pos0 = static_cast<uint32_t>(a + blk * kLanes + off);
-          if (off + 4 <= valid) {
+          if (off + 4 <= valid)
             q.offer4(v, pos0);
-          } else {
-            q.template offer<0>(v.x, pos0);
-            if (off + 1 < valid) q.template offer<1>(v.y, pos0 + 1);
-            if (off + 2 < valid) q.template offer<2>(v.z, pos0 + 2);
-          }
+          else
+            q.exact4(v, pos0, static_cast<int>(valid - off));
         }
       }
     }

@@ -20,127 +20,128 @@
 namespace tk {
 
 // ------------------------------------------------------------------ queues
-// Four register queues per thread.  Queue v keeps the best KB (key, index)
-// pairs offered to it, best-first.  Inside one queue indices arrive in
-// increasing order, so a strict comparison resolves ties by lowest index
-// without looking at the index.
+// Four register queues per thread.  Queue v keeps the best KB elements offered
+// to it, best-first, as (value, index) in the float domain; an empty slot holds
+// -inf with index kEmpty.  Elements reach a queue in increasing index order, so
+// "x ranks above slot s" needs no index comparison: with x neither NaN nor -inf
+// it is exactly the IEEE test x > val[s] (ties, -0 == +0 included, keep the
+// earlier element; a NaN slot is never beaten; an empty slot's -inf always is).
+// That fast update is branch-free: KB compares and 4 selects per slot.  NaN or
+// -inf values take the exact update, which compares order-preserving keys.
 //
-// k_b = 1: the queue is a running maximum kept in the float domain: thr[v] is
-// the best value so far (NaN before the first element), idx[v][0] its index,
-// and open[v] stays true until the queue holds a NaN (nothing can beat a NaN
-// that came first).  One offer costs a predicated compare and two selects:
-// the unordered test !(x <= thr) is true for x > thr, for a NaN x, and while
-// the queue is still empty; IEEE equality makes -0 tie +0 for free.
-// k_b > 1: keys are kept sorted in registers; thr[v] is the float value of the
-// worst kept entry (NaN while the queue is not full or when that entry is a
-// NaN), so the common case costs one float comparison.
+// Stored indices are "base" positions: queue v of a thread stores p - v for an
+// element at position p, so one base per float4 serves its four queues; the
+// true position is restored in store().
 template <int KB>
 struct Queues {
-  uint32_t key[4][KB];
+  float val[4][KB];
   uint32_t idx[4][KB];
-  float thr[4];
-  bool open[4];
 
-  static constexpr uint32_t kEmptyIdx = 0xffffffffu;
+  static constexpr uint32_t kEmpty = 0xffffffffu;
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
 #pragma unroll
       for (int s = 0; s < KB; ++s) {
-        key[v][s] = 0u;
-        idx[v][s] = kEmptyIdx;
+        val[v][s] = __int_as_float(0xff800000);
+        idx[v][s] = kEmpty;
       }
-      thr[v] = __uint_as_float(0x7fffffffu);
-      open[v] = true;
     }
   }
 
+  // Shift-insert given the monotone flags above[s] ("x ranks above slot s").
   template <int V>
-  __device__ __forceinline__ void take1(float x, uint32_t i) {
-    const bool p = open[V] && !(x <= thr[V]);
-    thr[V] = p ? x : thr[V];
-    idx[V][0] = p ? i : idx[V][0];
-    open[V] = open[V] && !(p && (x != x));
-  }
-
-  template <int V>
-  __device__ __forceinline__ void insert(float x, uint32_t i) {
-    const uint32_t kx = order_key(x);
-    if (kx <= key[V][KB - 1]) return;
-    bool placed = false;
+  __device__ __forceinline__ void place(const bool (&above)[KB], float x, uint32_t base) {
 #pragma unroll
     for (int s = KB - 1; s >= 0; --s) {
-      const int up_s = s > 0 ? s - 1 : 0;
-      const bool up = (s > 0) && (kx > key[V][up_s]);
-      const uint32_t nk = up ? key[V][up_s] : kx;
-      const uint32_t ni = up ? idx[V][up_s] : i;
-      if (!placed) {
-        key[V][s] = nk;
-        idx[V][s] = ni;
+      if (s > 0) {
+        const bool up = above[s > 0 ? s - 1 : 0];
+        const float vs = above[s] ? x : val[V][s];
+        const uint32_t is = above[s] ? base : idx[V][s];
+        val[V][s] = up ? val[V][s > 0 ? s - 1 : 0] : vs;
+        idx[V][s] = up ? idx[V][s > 0 ? s - 1 : 0] : is;
+      } else {
+        val[V][0] = above[0] ? x : val[V][0];
+        idx[V][0] = above[0] ? base : idx[V][0];
       }
-      placed = placed || !up;
     }
-    thr[V] = key[V][KB - 1] ? key_value(key[V][KB - 1]) : __uint_as_float(0x7fffffffu);
+  }
+
+  // x is neither NaN nor -inf.
+  template <int V>
+  __device__ __forceinline__ void insert_fast(float x, uint32_t base) {
+    bool above[KB];
+#pragma unroll
+    for (int s = 0; s < KB; ++s) above[s] = x > val[V][s];
+    place<V>(above, x, base);
+  }
+
+  // Any x (NaN ranks above +inf; all NaNs tie).
+  template <int V>
+  __device__ __forceinline__ void insert_exact(float x, uint32_t base) {
+    const uint32_t kx = order_key(x);
+    bool above[KB];
+#pragma unroll
+    for (int s = 0; s < KB; ++s)
+      above[s] = (idx[V][s] == kEmpty) || kx > order_key(val[V][s]);
+    place<V>(above, x, base);
   }
 
   template <int V>
-  __device__ __forceinline__ void offer(float x, uint32_t i) {
-    if (KB == 1) {
-      take1<V>(x, i);
-    } else if (!(x <= thr[V])) {
-      insert<V>(x, i);
-    }
+  __device__ __forceinline__ void offer(float x, uint32_t base) {
+    if (x > __int_as_float(0xff800000))
+      insert_fast<V>(x, base);
+    else
+      insert_exact<V>(x, base);
   }
 
-  // Four consecutive positions i0..i0+3 (one per queue).
-  __device__ __forceinline__ void offer4(const float4 x, uint32_t i0) {
-    offer<0>(x.x, i0);
-    offer<1>(x.y, i0 + 1);
-    offer<2>(x.z, i0 + 2);
-    offer<3>(x.w, i0 + 3);
+  __device__ __forceinline__ static bool special(const float4 x) {
+    const float ninf = __int_as_float(0xff800000);
+    return !(x.x > ninf) | !(x.y > ninf) | !(x.z > ninf) | !(x.w > ninf);
   }
 
-  // U float4 values x[u] at positions i0[u]..i0[u]+3, in increasing position
-  // order per queue; valid[u] false skips x[u].  For k_b > 1 the threshold tests
-  // of one queue are combined so that a queue whose U values all fail costs a
-  // single branch.
+  __device__ __forceinline__ void fast4(const float4 x, uint32_t base) {
+    insert_fast<0>(x.x, base);
+    insert_fast<1>(x.y, base);
+    insert_fast<2>(x.z, base);
+    insert_fast<3>(x.w, base);
+  }
+
+  __device__ __forceinline__ void exact4(const float4 x, uint32_t base, int valid = 4) {
+    if (valid > 0) insert_exact<0>(x.x, base);
+    if (valid > 1) insert_exact<1>(x.y, base);
+    if (valid > 2) insert_exact<2>(x.z, base);
+    if (valid > 3) insert_exact<3>(x.w, base);
+  }
+
+  // Positions base..base+3, one per queue.
+  __device__ __forceinline__ void offer4(const float4 x, uint32_t base) {
+    if (special(x))
+      exact4(x, base);
+    else
+      fast4(x, base);
+  }
+
+  // U float4 values at bases base[u] (increasing), all valid.  One NaN-keeping
+  // min over all 4U values decides whether any of them is NaN or -inf.
   template <int U>
-  __device__ __forceinline__ void offer_rows(const float4 (&x)[U], const uint32_t (&i0)[U],
-                                             const bool (&valid)[U]) {
-    if (KB == 1) {
+  __device__ __forceinline__ void offer_tile(const float4 (&x)[U], const uint32_t (&base)[U]) {
+    float m[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (valid[u]) offer4(x[u], i0[u]);
-      return;
-    }
-    bool any0 = false, any1 = false, any2 = false, any3 = false;
+    for (int u = 0; u < U; ++u)
+      m[u] = fmin_nan(fmin_nan(x[u].x, x[u].y), fmin_nan(x[u].z, x[u].w));
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      any0 |= valid[u] && !(x[u].x <= thr[0]);
-      any1 |= valid[u] && !(x[u].y <= thr[1]);
-      any2 |= valid[u] && !(x[u].z <= thr[2]);
-      any3 |= valid[u] && !(x[u].w <= thr[3]);
-    }
-    if (any0) {
+    for (int w = 1; w < U; w <<= 1)
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (valid[u]) offer<0>(x[u].x, i0[u]);
-    }
-    if (any1) {
+      for (int u = 0; u + w < U; u += 2 * w) m[u] = fmin_nan(m[u], m[u + w]);
+    const bool sp = !(m[0] > __int_as_float(0xff800000));
+    if (!sp) {
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (valid[u]) offer<1>(x[u].y, i0[u] + 1);
-    }
-    if (any2) {
+      for (int u = 0; u < U; ++u) fast4(x[u], base[u]);
+    } else {
 #pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (valid[u]) offer<2>(x[u].z, i0[u] + 2);
-    }
-    if (any3) {
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (valid[u]) offer<3>(x[u].w, i0[u] + 3);
+      for (int u = 0; u < U; ++u) exact4(x[u], base[u]);
     }
   }
 
@@ -151,12 +152,8 @@ struct Queues {
       uint64_t p = 0;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        if (w == v) {
-          if (KB == 1)
-            p = idx[w][0] != kEmptyIdx ? pack(order_key(thr[w]), idx[w][0]) : 0ull;
-          else
-            p = pack(key[w][s], idx[w][s]);
-        }
+        if (w == v && idx[w][s] != kEmpty)
+          p = pack(order_key(val[w][s]), idx[w][s] + static_cast<uint32_t>(w));
       }
       dst[s] = p;
     }
@@ -232,6 +229,135 @@ __device__ __forceinline__ void bitonic_desc(uint64_t* s, int N, int T) {
 
 enum ValueSource { kGatherInput = 0, kFromKey = 1 };
 
+// ------------------------------------------------------------------ register sort
+// Bitonic sort into descending order of the N = kThreads * EPT packed keys held
+// by the first kThreads threads, blocked (thread t holds elements t*EPT + j).
+// Exchanges inside a thread use registers, exchanges inside a warp use
+// shuffles, and only strides that cross warps go through shared memory (xchg,
+// N entries), so a 512-key sort needs 6 shared-memory rounds instead of 45.
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a > b ? b : a; }
+
+// One compare-exchange round of the network (SIZE, STRIDE fixed at compile time).
+template <int EPT, int SIZE, int STRIDE>
+__device__ __forceinline__ void bitonic_round(uint64_t (&v)[EPT], uint64_t* xchg) {
+  const int t = threadIdx.x;
+  if constexpr (STRIDE >= 32 * EPT) {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) xchg[t * EPT + j] = v[j];
+    group_sync(kThreads);
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = t * EPT + j;
+      const uint64_t o = xchg[e ^ STRIDE];
+      const bool keep_max = ((e & SIZE) == 0) == ((e & STRIDE) == 0);
+      v[j] = keep_max ? umax64(v[j], o) : umin64(v[j], o);
+    }
+    group_sync(kThreads);
+  } else if constexpr (STRIDE >= EPT) {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = t * EPT + j;
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, v[j], STRIDE / EPT);
+      const bool keep_max = ((e & SIZE) == 0) == ((e & STRIDE) == 0);
+      v[j] = keep_max ? umax64(v[j], o) : umin64(v[j], o);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      if ((j & STRIDE) == 0) {
+        const int jj = j | STRIDE;
+        const int e = t * EPT + j;
+        const uint64_t a = v[j], b = v[jj];
+        const bool desc = (e & SIZE) == 0;
+        v[j] = desc ? umax64(a, b) : umin64(a, b);
+        v[jj] = desc ? umin64(a, b) : umax64(a, b);
+      }
+    }
+  }
+  if constexpr (STRIDE > 1) bitonic_round<EPT, SIZE, STRIDE / 2>(v, xchg);
+}
+
+template <int EPT, int SIZE>
+__device__ __forceinline__ void bitonic_sizes(uint64_t (&v)[EPT], uint64_t* xchg) {
+  bitonic_round<EPT, SIZE, SIZE / 2>(v, xchg);
+  if constexpr (SIZE < kThreads * EPT) bitonic_sizes<EPT, SIZE * 2>(v, xchg);
+}
+
+template <int EPT>
+__device__ __forceinline__ void block_sort_desc(uint64_t (&v)[EPT], uint64_t* xchg) {
+  bitonic_sizes<EPT, 2>(v, xchg);
+}
+
+// Value of an output candidate: from its key, except that a zero or NaN is
+// re-read from the input row so that -0.0 and NaN payloads keep their bits.
+template <int VS>
+__device__ __forceinline__ float candidate_value(uint64_t p, const float* xrow) {
+  float v = key_value(packed_key(p));
+  if (VS == 0 && (v == 0.0f || v != v)) v = __ldg(xrow + packed_idx(p));
+  return v;
+}
+
+template <int EPT, int VS>
+__device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, const float* xrow,
+                                                  float* ov, int32_t* oi) {
+  constexpr int N = kThreads * EPT;
+  const int t = threadIdx.x;
+  uint64_t v[EPT];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = t * EPT + j;
+    v[j] = e < C ? cand[e] : 0ull;
+  }
+  group_sync(kThreads);  // cand is reused as the exchange buffer
+  block_sort_desc<EPT>(v, cand);
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = t * EPT + j;
+    if (e < k) {
+      if (v[j]) {
+        ov[e] = candidate_value<VS>(v[j], xrow);
+        oi[e] = static_cast<int32_t>(packed_idx(v[j]));
+      } else {
+        ov[e] = __int_as_float(0xff800000);
+        oi[e] = -1;
+      }
+    }
+  }
+  for (int e = N + t; e < k; e += kThreads) {
+    ov[e] = __int_as_float(0xff800000);
+    oi[e] = -1;
+  }
+  group_sync(kThreads);
+}
+
+// Candidate buffer entries the register sort needs for C candidates.
+__host__ __device__ __forceinline__ int sort_capacity(int C) {
+  int n = kThreads;
+  while (n < C) n <<= 1;
+  return n;
+}
+
+template <ValueSource VS>
+__device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const float* xrow,
+                                             float* ov, int32_t* oi, int T);
+
+// Stage 2 for the streaming kernels (kThreads threads): up to 8 keys per
+// thread are sorted in registers; larger candidate sets use the shared-memory
+// network.
+template <ValueSource VS>
+__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const float* xrow,
+                                                  float* ov, int32_t* oi) {
+  const int ept = sort_capacity(C) / kThreads;
+  switch (ept) {
+    case 1: finalize_row_regs<1, VS>(cand, C, k, xrow, ov, oi); break;
+    case 2: finalize_row_regs<2, VS>(cand, C, k, xrow, ov, oi); break;
+    case 4: finalize_row_regs<4, VS>(cand, C, k, xrow, ov, oi); break;
+    case 8: finalize_row_regs<8, VS>(cand, C, k, xrow, ov, oi); break;
+    default: finalize_row<VS>(cand, C, k, xrow, ov, oi, kThreads); break;
+  }
+}
+
 // cand[0..C) holds the Stage-1 candidates (0 = empty).  Sorts them best-first
 // and writes the first k (Stage 2: only the k best survive when C > k), padding
 // with -inf / -1.  Values either come from the input row (exact input bits)
@@ -291,7 +417,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
   if (a == 0 && len == rs.n) {
     merge_lanes<KB>(lanebuf, b, 0, cand, T);
     group_sync(T);
-    finalize_row<VS>(cand, C, k, xrow, ov, oi, T);
+    finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
     return;
   }
   const int64_t row0 = r * rs.n;
@@ -330,7 +456,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
     for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
   }
   group_sync(T);
-  finalize_row<VS>(cand, C, k, xrow, ov, oi, T);
+  finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
   if (threadIdx.x == 0) rs.tickets[r] = 0u;  // leave the workspace zeroed
 }
 

@@ -173,7 +173,10 @@ int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, 
   const int64_t cap = static_cast<int64_t>(sms) * per_sm;
   const int64_t units = E / align;
   int64_t G;
-  if (rows <= cap && (rows >= sms || rows * min_piece >= E)) {
+#ifndef TOPK_GRID_ONE_ROW_PER_CTA
+#define TOPK_GRID_ONE_ROW_PER_CTA 1
+#endif
+  if (TOPK_GRID_ONE_ROW_PER_CTA && rows <= cap && (rows >= sms || rows * min_piece >= E)) {
     G = rows;  // one row per CTA: no row is split
   } else {
     G = std::min<int64_t>(cap, std::max<int64_t>(1, (E + min_piece - 1) / min_piece));
@@ -186,7 +189,7 @@ int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, 
 template <int KB>
 int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
   const int C = b * KB;
-  pl->cand_cap = host_next_pow2(C);
+  pl->cand_cap = sort_capacity(C);
   pl->align = fast ? 4 : 1;
   pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap}, 2) : 0;
   int per_sm = 0;
@@ -225,7 +228,7 @@ int plan_select(bool fast, int64_t rows, int64_t n, int b, int kb, const DeviceI
 template <int KB, int D>
 int plan_score_kd(int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
   const int C = b * KB;
-  pl->cand_cap = host_next_pow2(C);
+  pl->cand_cap = sort_capacity(C);
   pl->align = 1;
   pl->stages = fit_stages(ScoreSmem{0, KB, pl->cand_cap}, 2);
   ScoreSmem L{pl->stages, KB, pl->cand_cap};
