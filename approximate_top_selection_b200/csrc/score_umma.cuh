@@ -1,0 +1,460 @@
+// score_umma.cuh -- fused link-prediction selector: S = Q K^T on the 5th-gen
+// tensor cores (tcgen05.mma, bf16 in, fp32 accumulators in TMEM), each score
+// pushed straight into its bucket queue by the epilogue; S never reaches HBM.
+//
+// Application: "Approximate Top-k for Increased Parallelism" (arXiv 2412.04358),
+// "Core claim" and Fig. 4 (right): knowledge-graph link prediction scores every
+// query against millions of entities and keeps the top k = 100 with k_b = 1.
+// Selection: the bucketed two-stage top-k of "What carries the argument".
+//
+// Work unit = (128 queries, group of 8 buckets).  Entity e = t*b + j belongs to
+// bucket j, so a unit walks the entities t*b + 8g + jj (jj < 8) for all t.  The
+// TMA engine fetches them as a 3-D box {64 d, 8 jj, 32 t} of the key matrix
+// viewed as [T][b][d]: 256 key rows of 128 B with the 128-byte swizzle, which is
+// exactly a K-major UMMA B operand.  Accumulator column c of a 128 x 256 tile
+// is then entity (t0 + c/8)*b + 8g + c%8, i.e. bucket 8g + c%8, and each
+// epilogue thread (one query row) keeps only 8 bucket queues in registers.
+//
+// Warp roles (320 threads): warp 0 issues TMA loads (Q tile once per unit, key
+// stages through a ring), warp 1 owns TMEM (512 columns = two 128x256 fp32
+// accumulators) and issues the MMAs from one thread, warps 2..9 drain TMEM
+// (tcgen05.ld) and update the queues: two warps per TMEM lane quarter, one per
+// half of the 256 columns.  Per-unit results (top-k_b per bucket and column half)
+// go to the workspace; umma_finish merges the halves and runs Stage 2.
+//
+// The units of one bucket group are consecutive, so the 8 query tiles that read
+// the same key rows run at about the same time and share them through L2.
+#pragma once
+
+#include <cuda.h>
+
+#include "select_core.cuh"
+
+namespace tk {
+
+constexpr int kUmmaM = 128;            // queries per tile (TMEM lanes)
+constexpr int kUmmaN = 256;            // entities per tile (accumulator columns)
+constexpr int kUmmaGroup = 8;          // buckets per unit
+constexpr int kUmmaTPerTile = kUmmaN / kUmmaGroup;  // 32 stripes per tile
+constexpr int kUmmaChunkBytes = 16384;              // 128 rows x 64 bf16 (A chunk)
+constexpr int kUmmaStageBytes = 32768;              // 256 rows x 64 bf16 (B stage)
+constexpr int kUmmaStages = 4;
+constexpr int kUmmaThreads = 320;
+constexpr int kUmmaEpiWarps = 8;
+
+struct UmmaArgs {
+  int64_t rows, n;   // queries, entities
+  int b, T;          // buckets, stripes (n = T * b)
+  int mtiles, groups, tiles_per_unit, units;
+  float* out_scores;  // nullable [rows][n]
+  uint64_t* cand;     // [rows][b][2][KB]
+};
+
+template <int D>
+struct UmmaSmem {
+  static constexpr int kChunks = D / 64;
+  static constexpr size_t a_bytes = static_cast<size_t>(kChunks) * kUmmaChunkBytes;
+  static constexpr size_t b_bytes = static_cast<size_t>(kUmmaStages) * kUmmaStageBytes;
+  static constexpr size_t bar_bytes = 1024;
+  static constexpr size_t total = 1024 /* alignment slack */ + a_bytes + b_bytes + bar_bytes;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* tm, int c0, int c1,
+                                            int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile with the 128-byte swizzle:
+// rows of 128 B, 8-row groups 1024 B apart (stride byte offset), sm_100 form.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                   // leading byte offset (unused here)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;           // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                   // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                   // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16: D = f32, A = B = bf16, both K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ queues
+// NQ bucket queues of KB entries (value domain, as Queues in select_core.cuh),
+// storing true entity indices.
+template <int NQ, int KB>
+struct BucketQueues {
+  float val[NQ][KB];
+  uint32_t idx[NQ][KB];
+  static constexpr uint32_t kEmpty = 0xffffffffu;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int s = 0; s < KB; ++s) {
+        val[q][s] = __int_as_float(0xff800000);
+        idx[q][s] = kEmpty;
+      }
+  }
+
+  template <int Q>
+  __device__ __forceinline__ void place(const bool (&above)[KB], float x, uint32_t i) {
+#pragma unroll
+    for (int s = KB - 1; s >= 0; --s) {
+      if (s > 0) {
+        const bool up = above[s > 0 ? s - 1 : 0];
+        const float vs = above[s] ? x : val[Q][s];
+        const uint32_t is = above[s] ? i : idx[Q][s];
+        val[Q][s] = up ? val[Q][s > 0 ? s - 1 : 0] : vs;
+        idx[Q][s] = up ? idx[Q][s > 0 ? s - 1 : 0] : is;
+      } else {
+        val[Q][0] = above[0] ? x : val[Q][0];
+        idx[Q][0] = above[0] ? i : idx[Q][0];
+      }
+    }
+  }
+
+  template <int Q>
+  __device__ __forceinline__ void insert_fast(float x, uint32_t i) {
+    bool above[KB];
+#pragma unroll
+    for (int s = 0; s < KB; ++s) above[s] = x > val[Q][s];
+    place<Q>(above, x, i);
+  }
+
+  template <int Q>
+  __device__ __forceinline__ void insert_exact(float x, uint32_t i) {
+    const uint32_t kx = order_key(x);
+    bool above[KB];
+#pragma unroll
+    for (int s = 0; s < KB; ++s) above[s] = (idx[Q][s] == kEmpty) || kx > order_key(val[Q][s]);
+    place<Q>(above, x, i);
+  }
+};
+
+// Feeds the 32 scores of one tcgen05.ld (columns c0 .. c0+31 of the tile, c0 a
+// multiple of 32, so column r belongs to queue r % 8 and stripe c0/8 + r/8).
+template <int KB>
+__device__ __forceinline__ void umma_feed(BucketQueues<kUmmaGroup, KB>& q, const uint32_t (&r)[32],
+                                          int c0, int t0, int T, uint32_t b, uint32_t jbase,
+                                          int64_t row, int64_t rows, int64_t n, float* out_scores) {
+  float m = __uint_as_float(r[0]);
+#pragma unroll
+  for (int i = 1; i < 32; ++i) m = fmin_nan(m, __uint_as_float(r[i]));
+  const bool special = !(m > __int_as_float(0xff800000));
+  const int tfirst = t0 + c0 / kUmmaGroup;
+  const bool full = tfirst + 4 <= T;
+  if (out_scores != nullptr && row < rows) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = tfirst + i / kUmmaGroup;
+      if (t < T)
+        out_scores[row * n + static_cast<int64_t>(t) * b + jbase + (i % kUmmaGroup)] =
+            __uint_as_float(r[i]);
+    }
+  }
+#define TK_FEED_ONE(I)                                                                    \
+  {                                                                                       \
+    const int t = tfirst + (I) / kUmmaGroup;                                              \
+    const uint32_t e = static_cast<uint32_t>(t) * b + jbase + ((I) % kUmmaGroup);          \
+    if (full || t < T) {                                                                  \
+      if (special)                                                                        \
+        q.template insert_exact<(I) % kUmmaGroup>(__uint_as_float(r[I]), e);              \
+      else                                                                                \
+        q.template insert_fast<(I) % kUmmaGroup>(__uint_as_float(r[I]), e);               \
+    }                                                                                     \
+  }
+  TK_FEED_ONE(0) TK_FEED_ONE(1) TK_FEED_ONE(2) TK_FEED_ONE(3) TK_FEED_ONE(4) TK_FEED_ONE(5)
+  TK_FEED_ONE(6) TK_FEED_ONE(7) TK_FEED_ONE(8) TK_FEED_ONE(9) TK_FEED_ONE(10) TK_FEED_ONE(11)
+  TK_FEED_ONE(12) TK_FEED_ONE(13) TK_FEED_ONE(14) TK_FEED_ONE(15) TK_FEED_ONE(16)
+  TK_FEED_ONE(17) TK_FEED_ONE(18) TK_FEED_ONE(19) TK_FEED_ONE(20) TK_FEED_ONE(21)
+  TK_FEED_ONE(22) TK_FEED_ONE(23) TK_FEED_ONE(24) TK_FEED_ONE(25) TK_FEED_ONE(26)
+  TK_FEED_ONE(27) TK_FEED_ONE(28) TK_FEED_ONE(29) TK_FEED_ONE(30) TK_FEED_ONE(31)
+#undef TK_FEED_ONE
+}
+
+template <int KB, int D>
+__global__ void __launch_bounds__(kUmmaThreads, 1)
+    score_select_umma(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      UmmaArgs p) {
+  using L = UmmaSmem<D>;
+  constexpr int kChunks = L::kChunks;
+  constexpr uint32_t kIdesc = umma_idesc_bf16(kUmmaM, kUmmaN);
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte alignment for the swizzled operand tiles.
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  unsigned char* a_tile = smem;
+  unsigned char* b_ring = smem + L::a_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::a_bytes + L::b_bytes);
+  uint64_t* a_full = bars + 0;
+  uint64_t* a_empty = bars + 1;
+  uint64_t* full_b = bars + 2;                   // [kUmmaStages]
+  uint64_t* empty_b = bars + 2 + kUmmaStages;    // [kUmmaStages]
+  uint64_t* acc_full = bars + 2 + 2 * kUmmaStages;   // [2]
+  uint64_t* acc_empty = bars + 4 + 2 * kUmmaStages;  // [2]
+  uint64_t* mma_done = bars + 6 + 2 * kUmmaStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7 + 2 * kUmmaStages);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(a_full, 1);
+    mbar_init(a_empty, 1);
+    for (int s = 0; s < kUmmaStages; ++s) {
+      mbar_init(full_b + s, 1);
+      mbar_init(empty_b + s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(acc_full + s, 1);
+      mbar_init(acc_empty + s, kUmmaEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      int64_t bt = 0;  // key stages issued
+      int iu = 0;
+      for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x, ++iu) {
+        const int m = u % p.mtiles, g = u / p.mtiles;
+        if (iu > 0 && !mbar_wait_or_abort(a_empty, static_cast<uint32_t>((iu - 1) & 1), abort_flag))
+          break;
+        mbar_expect_tx(a_full, static_cast<uint32_t>(L::a_bytes));
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_2d(a_tile + c * kUmmaChunkBytes, &tmQ, c * 64, m * kUmmaM, a_full);
+        bool ok = true;
+        for (int tile = 0; tile < p.tiles_per_unit && ok; ++tile) {
+          for (int c = 0; c < kChunks; ++c) {
+            if (bt >= kUmmaStages && !mbar_wait_or_abort(empty_b + st, ph ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(full_b + st, kUmmaStageBytes);
+            tma_load_3d(b_ring + st * kUmmaStageBytes, &tmK, c * 64, g * kUmmaGroup,
+                        tile * kUmmaTPerTile, full_b + st);
+            ++bt;
+            if (++st == kUmmaStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {
+        // Let the copies already issued land before the CTA can go away.
+        for (int64_t x = (bt > kUmmaStages ? bt - kUmmaStages : 0); x < bt; ++x)
+          mbar_wait(full_b + (x % kUmmaStages), static_cast<uint32_t>((x / kUmmaStages) & 1),
+                    100000000ull);
+        if (iu > 0) mbar_wait(a_full, static_cast<uint32_t>((iu - 1) & 1), 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      int64_t tg = 0;  // tiles issued by this CTA
+      int iu = 0;
+      const uint32_t a_base = smem_addr(a_tile), b_base = smem_addr(b_ring);
+      for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x, ++iu) {
+        if (!mbar_wait_or_abort(a_full, static_cast<uint32_t>(iu & 1), abort_flag)) break;
+        bool ok = true;
+        for (int tile = 0; tile < p.tiles_per_unit && ok; ++tile, ++tg) {
+          const int buf = static_cast<int>(tg & 1);
+          if (tg >= 2 &&
+              !mbar_wait_or_abort(acc_empty + buf, static_cast<uint32_t>(((tg >> 1) - 1) & 1),
+                                  abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + static_cast<uint32_t>(buf * kUmmaN);
+          for (int c = 0; c < kChunks; ++c) {
+            if (!mbar_wait_or_abort(full_b + st, ph, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = umma_desc_sw128(a_base + c * kUmmaChunkBytes + kk * 32);
+              const uint64_t bd = umma_desc_sw128(b_base + st * kUmmaStageBytes + kk * 32);
+              umma_bf16(d_tmem, ad, bd, kIdesc, (c | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(empty_b + st);  // the stage is free once these MMAs are done
+            if (++st == kUmmaStages) {
+              st = 0;
+              ph ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(acc_full + buf);
+        }
+        if (!ok) break;
+        umma_commit(a_empty);
+      }
+      // Every MMA this thread issued has completed before TMEM is released.
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, 1000000000ull);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 2;
+    const int quarter = warp & 3;            // TMEM lanes this warp may read
+    const int half = ew >> 2;                // which 128 columns of the tile
+    const int64_t row_in_tile = quarter * 32 + lane;
+    BucketQueues<kUmmaGroup, KB> q;
+    int64_t tg = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+      const int m = u % p.mtiles, g = u / p.mtiles;
+      const int64_t row = static_cast<int64_t>(m) * kUmmaM + row_in_tile;
+      const uint32_t jbase = static_cast<uint32_t>(g * kUmmaGroup);
+      q.reset();
+      bool ok = true;
+      for (int tile = 0; tile < p.tiles_per_unit; ++tile, ++tg) {
+        const int buf = static_cast<int>(tg & 1);
+        ok = __any_sync(0xffffffffu,
+                        !*abort_flag && mbar_wait_or_abort(acc_full + buf,
+                                                           static_cast<uint32_t>((tg >> 1) & 1),
+                                                           abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const int t0 = tile * kUmmaTPerTile;
+        const uint32_t taddr =
+            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * kUmmaN);
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+          const int c0 = half * 128 + i * 32;
+          uint32_t r[32];
+          tmem_ld_x32(taddr + static_cast<uint32_t>(c0), r);
+          if (i == 3) {
+            // Everything of this buffer is in registers: hand it back to the MMA.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty + buf);
+          }
+          umma_feed<KB>(q, r, c0, t0, p.T, static_cast<uint32_t>(p.b), jbase, row, p.rows, p.n,
+                        p.out_scores);
+        }
+      }
+      if (!ok) break;
+      if (row < p.rows) {
+        uint64_t* dst = p.cand + ((static_cast<size_t>(row) * p.b + jbase) * 2 + half) * KB;
+#pragma unroll
+        for (int j = 0; j < kUmmaGroup; ++j)
+#pragma unroll
+          for (int s = 0; s < KB; ++s)
+            dst[static_cast<size_t>(j) * 2 * KB + s] =
+                q.idx[j][s] != BucketQueues<kUmmaGroup, KB>::kEmpty
+                    ? pack(order_key(q.val[j][s]), q.idx[j][s])
+                    : 0ull;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
+                 : "memory");
+  }
+}
+
+// Stage 2 of the tensor-core path: per query, the top-k_b of each bucket over
+// the two column halves, then the exact top-k of the b*k_b candidates.
+template <int KB>
+__global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64_t rows, int b,
+                                                        int k, float* out_vals, int32_t* out_idx) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem);
+  const int64_t r = blockIdx.x;
+  for (int j = threadIdx.x; j < b; j += kThreads) {
+    uint64_t best[KB];
+#pragma unroll
+    for (int s = 0; s < KB; ++s) best[s] = 0;
+    uint64_t* src = cand_ws + (static_cast<size_t>(r) * b + j) * 2 * KB;
+#pragma unroll
+    for (int s = 0; s < 2 * KB; ++s) {
+      keep_best<KB>(best, src[s]);
+      src[s] = 0ull;  // leave the workspace zeroed for the next call
+    }
+#pragma unroll
+    for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
+  }
+  group_sync(kThreads);
+  finalize_row_fast<kFromKey>(cand, b * KB, k, nullptr, out_vals + r * k, out_idx + r * k);
+}
+
+}  // namespace tk

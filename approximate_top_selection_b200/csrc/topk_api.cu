@@ -1,5 +1,7 @@
 // topk_api.cu -- the C ABI (include/topk_b200.h): argument checks, launch
 // plans and kernel launches.  All device work lives in the included kernels.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -11,6 +13,7 @@
 #include "bucket_select.cuh"
 #include "exact_topk.cuh"
 #include "score_gemv.cuh"
+#include "score_umma.cuh"
 
 namespace tk {
 namespace {
@@ -328,6 +331,102 @@ int launch_score_k(int d, const Plan& pl, const ScoreArgs& a, cudaStream_t st) {
   return launch_score_kd<KB, 256>(pl, a, st);
 }
 
+// ---------------------------------------------------------------- tensor-core path
+// Fused link-prediction selector on tcgen05 (score_umma.cuh): one key matrix
+// shared by all rows, b a multiple of 8 dividing n, enough rows to fill M tiles.
+constexpr int64_t kUmmaMinRows = 32;
+
+bool umma_eligible(int64_t rows, int64_t n, int64_t kstride, int b, int d) {
+  return kstride == 0 && rows >= kUmmaMinRows && (b % kUmmaGroup) == 0 && (n % b) == 0 &&
+         (d == 128 || d == 256) && rows <= (1LL << 31) - 1;
+}
+
+size_t umma_workspace(int64_t rows, int b, int kb) {
+  return static_cast<size_t>(rows) * b * 2 * kb * 8;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
+  std::lock_guard<std::mutex> lk(g_encode_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || fn == nullptr)
+      return TOPK_ECUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = g_encode;
+  return TOPK_OK;
+}
+
+template <int KB, int D>
+int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n, int b, int k,
+                   float* out_vals, int32_t* out_idx, float* out_scores, void* ws,
+                   const DeviceInfo& dev, cudaStream_t st) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+  int rc = tensor_map_encoder(&encode);
+  if (rc) return rc;
+  const int64_t T = n / b;
+  CUtensorMap tmQ, tmK;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64, kUmmaM};
+    const cuuint32_t es[2] = {1, 1};
+    if (encode(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return TOPK_ECUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(b),
+                                static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(b) * D * 2};
+    const cuuint32_t box[3] = {64, kUmmaGroup, kUmmaTPerTile};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (encode(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(K), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return TOPK_ECUDA;
+  }
+  UmmaArgs a;
+  a.rows = rows;
+  a.n = n;
+  a.b = b;
+  a.T = static_cast<int>(T);
+  a.mtiles = static_cast<int>((rows + kUmmaM - 1) / kUmmaM);
+  a.groups = b / kUmmaGroup;
+  a.tiles_per_unit = static_cast<int>((T + kUmmaTPerTile - 1) / kUmmaTPerTile);
+  a.units = a.mtiles * a.groups;
+  a.out_scores = out_scores;
+  a.cand = static_cast<uint64_t*>(ws);
+  const size_t smem = UmmaSmem<D>::total;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  if ((rc = prepare_kernel(score_select_umma<KB, D>))) return rc;
+  if ((rc = prepare_kernel(umma_finish<KB>))) return rc;
+  const int grid = std::min(a.units, dev.sms);
+  clear_launch_error();
+  score_select_umma<KB, D><<<grid, kUmmaThreads, smem, st>>>(tmQ, tmK, a);
+  if ((rc = launch_status())) return rc;
+  const size_t fsmem = static_cast<size_t>(sort_capacity(b * KB)) * 8;
+  umma_finish<KB><<<static_cast<unsigned>(rows), kThreads, fsmem, st>>>(
+      a.cand, rows, b, k, out_vals, out_idx);
+  return launch_status();
+}
+
+template <int KB>
+int launch_umma_k(int d, const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n, int b,
+                  int k, float* ov, int32_t* oi, float* os, void* ws, const DeviceInfo& dev,
+                  cudaStream_t st) {
+  if (d == 128) return launch_umma_kd<KB, 128>(q, rows, K, n, b, k, ov, oi, os, ws, dev, st);
+  return launch_umma_kd<KB, 256>(q, rows, K, n, b, k, ov, oi, os, ws, dev, st);
+}
+
 // ---------------------------------------------------------------- no-alloc scratch
 // Built-in scratch of topk_bucketed_noalloc.  In host code this name is only a
 // stand-in for the symbol: the device address is looked up per device.
@@ -396,7 +495,9 @@ size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int k
   if (op == TOPK_OP_SCORE) {
     if (kLanes % b) return 0;
     if (plan_score(rows, n, b, kb, d, dev, &pl)) return 0;
-    return pl.workspace();
+    size_t need = pl.workspace();
+    if (umma_eligible(rows, n, 0, b, d)) need = std::max(need, umma_workspace(rows, b, kb));
+    return need;
   }
   return 0;
 }
@@ -499,6 +600,18 @@ int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_
   if (!aligned16(q) || !aligned16(K) || (k_batch_stride % 8) != 0) return TOPK_EINVAL;
   DeviceInfo dev;
   if ((rc = current_device_info(&dev))) return rc;
+  cudaStream_t sst = static_cast<cudaStream_t>(stream);
+  if (umma_eligible(rows, n, k_batch_stride, b, d)) {
+    const size_t need = umma_workspace(rows, b, kb);
+    if (!workspace || workspace_bytes < need) return TOPK_EWORKSPACE;
+    if (!aligned16(workspace)) return TOPK_EINVAL;
+    switch (kb) {
+      case 1: return launch_umma_k<1>(d, q, rows, K, n, b, k, out_vals, out_idx, out_scores, workspace, dev, sst);
+      case 2: return launch_umma_k<2>(d, q, rows, K, n, b, k, out_vals, out_idx, out_scores, workspace, dev, sst);
+      case 3: return launch_umma_k<3>(d, q, rows, K, n, b, k, out_vals, out_idx, out_scores, workspace, dev, sst);
+      default: return launch_umma_k<4>(d, q, rows, K, n, b, k, out_vals, out_idx, out_scores, workspace, dev, sst);
+    }
+  }
   Plan pl;
   if ((rc = plan_score(rows, n, b, kb, d, dev, &pl))) return rc;
   if (plan_needs_workspace(pl, rows, n)) {

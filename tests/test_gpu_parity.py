@@ -211,9 +211,19 @@ def check_scores(q: torch.Tensor, K: torch.Tensor, k, b, kb, oracle_mod, rows_su
     """q, K on the device.  Returns the GPU outputs after all checks."""
     v, i, s = atk.score_topk(q, K, k, b, kb, return_scores=True)
     torch.cuda.synchronize()
-    v, i, s = v.cpu().numpy(), i.cpu().numpy(), s.cpu().numpy()
     rows = q.shape[0]
     sub = np.arange(rows) if rows_subset is None else np.asarray(rows_subset)
+    if rows_subset is not None:  # copy back only the sampled rows
+        keep = torch.as_tensor(sub, device=s.device)
+        v = torch.zeros_like(v).index_copy_(0, keep, v[keep])
+        i = torch.zeros_like(i).index_copy_(0, keep, i[keep])
+        s = s[keep]
+        s_full = np.zeros((rows, s.shape[1]), np.float32)
+        s_full[sub] = s.cpu().numpy()
+        s = s_full
+    else:
+        s = s.cpu().numpy()
+    v, i = v.cpu().numpy(), i.cpu().numpy()
     # (1) the selection on the GPU's own scores is the oracle's, bit for bit
     ov, oi = oracle_mod.bucketed(s[sub], k, b, kb)
     assert np.array_equal(i[sub], oi) and same_bits(v[sub], ov)
@@ -275,3 +285,34 @@ def test_decode_config_full(oracle_mod):
     """16 x 32 rows, 32768 keys of d=128: sampled rows against the oracle."""
     q, K = inputs.decode_inputs(16, 32, 32768, 128, inputs.SEEDS["decode"], device=DEV)
     check_scores(q, K, 512, 256, 2, oracle_mod, rows_subset=[0, 1, 100, 255, 256, 400, 511])
+
+
+# ------------------------------------------------------------------ tensor-core scoring
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb", [1, 2, 4])
+def test_link_umma_shapes(oracle_mod, d, kb):
+    """Shared key matrix, b | n and >= 32 queries: the tcgen05 path.  Ragged
+    query tiles (not a multiple of 128) and stripe counts that are not a
+    multiple of the 32-stripe tile are included."""
+    for (rows, T, b, k) in [(32, 32, 64, 50), (200, 37, 64, 100), (130, 70, 256, 300)]:
+        Q, K = inputs.link_inputs(rows, T * b, d, 31 + rows + d + kb)
+        check_scores(Q.to(DEV), K.to(DEV), k, b, kb, oracle_mod)
+
+
+def test_link_umma_special_values(oracle_mod):
+    """Scores that are +-inf or NaN (from inf / NaN inputs) take the exact
+    queue update: the selection on the GPU's scores is still the oracle's."""
+    Q, K = inputs.link_inputs(64, 64 * 32, 128, 41)
+    K[5, :] = float("inf")
+    K[77, 3] = float("nan")
+    K[100, :] = -float("inf")
+    v, i, s = atk.score_topk(Q.to(DEV), K.to(DEV), 40, 64, 2, return_scores=True)
+    ov, oi = oracle_mod.bucketed(s.cpu().numpy(), 40, 64, 2)
+    assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+
+
+def test_link_config_full(oracle_mod):
+    """1024 queries x 2^20 entities, d = 256, k = 100, b = 1024, k_b = 1:
+    sampled query rows against the fp64 oracle."""
+    Q, K = inputs.link_inputs(1024, 1 << 20, 256, inputs.SEEDS["link"], device=DEV)
+    check_scores(Q, K, 100, 1024, 1, oracle_mod, rows_subset=[0, 127, 128, 500, 1023])
