@@ -46,8 +46,9 @@ CONFIGS = {
     "decode": dict(kind="score", batch=16, heads=32, n=32768, d=128, k=512, b=256, kb=2),
     "vocab": dict(kind="select", rows=256, n=131072, k=50, b=512, kb=1, dist="vocab"),
     "link": dict(kind="score", queries=1024, n=1 << 20, d=256, k=100, b=1024, kb=1),
-    # a quarter of the decode rows (1 GiB of keys): the case profiled with ncu --set full
+    # reduced cases profiled with ncu --set full (inputs still larger than L2)
     "decode-quarter": dict(kind="score", batch=4, heads=32, n=32768, d=128, k=512, b=256, kb=2),
+    "link-quarter": dict(kind="score", queries=1024, n=1 << 18, d=256, k=100, b=1024, kb=1),
 }
 for _b in (128, 256, 512):
     for _kb in (1, 2, 4):
@@ -338,6 +339,34 @@ def run_ours(args, world, rank, local):
     return line
 
 
+def _source_hash() -> str:
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "approximate_top_selection_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels
+    have not changed since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.md")
+    if not os.path.exists(path):
+        return None
+    cur = _source_hash()
+    for line in open(path):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[0] == workload and cells[2] == cur:
+            try:
+                return int(cells[3])
+            except ValueError:
+                return None
+    return None
+
+
 def _roofline(w: Workload, ms_step: float, achieved_gbs: float, hbm: float, peak_src: str):
     c = w.cfg
     if _uses_tensor_cores(c):
@@ -345,10 +374,10 @@ def _roofline(w: Workload, ms_step: float, achieved_gbs: float, hbm: float, peak
         tf = flops / (ms_step * 1e-3) / 1e12
         peak, src = _tensor_peak()
         return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                "frac": tf / peak, "traffic": None, "kernel": _kernel_name(c),
+                "frac": tf / peak, "traffic": _traffic(w.name), "kernel": _kernel_name(c),
                 "flops_per_step": flops, "peak_source": src}
     return {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-            "frac": achieved_gbs / hbm, "traffic": None, "kernel": _kernel_name(c),
+            "frac": achieved_gbs / hbm, "traffic": _traffic(w.name), "kernel": _kernel_name(c),
             "peak_source": peak_src + " hbm_gbs"}
 
 
