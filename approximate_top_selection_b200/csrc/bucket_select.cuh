@@ -35,15 +35,90 @@ struct SelectArgs {
 
 // Shared-memory layout of the selection kernels (bytes).
 struct SelectSmem {
-  int stages, kb, cand_cap;
+  int stages, kb, cand_cap, nl;  // nl: register queues (lanes) per CTA
   __host__ __device__ size_t ring_bytes() const { return static_cast<size_t>(stages) * kTile * 4; }
-  __host__ __device__ size_t lane_bytes() const { return static_cast<size_t>(kLanes) * kb * 8; }
-  __host__ __device__ size_t cand_bytes() const { return static_cast<size_t>(cand_cap) * 8; }
+  __host__ __device__ size_t lane_bytes() const { return static_cast<size_t>(nl) * kb * 8; }
+  __host__ __device__ size_t cand_bytes() const {
+    return static_cast<size_t>(cand_cap) * 8 + kStage2Extra;
+  }
   __host__ __device__ size_t bar_bytes() const { return 16 * static_cast<size_t>(stages) + 16; }
   __host__ __device__ size_t total() const {
     return ring_bytes() + lane_bytes() + cand_bytes() + bar_bytes();
   }
 };
+
+// k_b > 2: one tile (c valid floats at row positions pos_tile ...) for the
+// queues of this thread: element u sits at tile offset t + 256 u and feeds
+// queue u mod nq.  Each element is first compared with its queue's worst
+// entry; only the survivors -- typically a few per thread per tile once the
+// queues have filled -- go through the sorted insert, re-read from shared
+// memory, so a warp pays for its busiest thread's survivors rather than for
+// every element.  A tile holding NaN or -inf takes the exact update instead.
+template <int KB>
+__device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const float* tile, uint32_t c,
+                                                   uint32_t pos_tile, int nq) {
+  constexpr int U = kTile / kThreads;  // 32 elements per thread
+  const int t = threadIdx.x;
+  float x[U];
+  float m = __int_as_float(0x7f800000);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const bool valid = static_cast<uint32_t>(t + kThreads * u) < c;
+    x[u] = valid ? tile[t + kThreads * u] : __int_as_float(0x7f800000);
+    m = fmin_nan(m, x[u]);
+  }
+  const uint32_t base = pos_tile + static_cast<uint32_t>(t);
+  if (!(m > __int_as_float(0xff800000))) {
+    // NaN or -inf somewhere in this thread's elements: exact update, in order.
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (static_cast<uint32_t>(t + kThreads * u) >= c) continue;
+      const uint32_t pos = base + static_cast<uint32_t>(kThreads * u);
+      const int qq = u % nq;
+      if (qq == 0) q.template insert_exact<0>(x[u], pos);
+      if (qq == 1) q.template insert_exact<1>(x[u], pos - 1);
+      if (qq == 2) q.template insert_exact<2>(x[u], pos - 2);
+      if (qq == 3) q.template insert_exact<3>(x[u], pos - 3);
+    }
+    return;
+  }
+  // Survivor masks per queue (queue of element u is u mod nq; nq is 1, 2 or 4).
+  uint32_t mask[4] = {0u, 0u, 0u, 0u};
+  const float thr[4] = {q.val[0][KB - 1], q.val[1][KB - 1], q.val[2][KB - 1], q.val[3][KB - 1]};
+  if (nq == 1) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      mask[0] |= (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[0]) ? (1u << u) : 0u;
+  } else if (nq == 2) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      mask[u & 1] |=
+          (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[u & 1]) ? (1u << u) : 0u;
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      mask[u & 3] |=
+          (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[u & 3]) ? (1u << u) : 0u;
+  }
+#define TK_SURVIVORS(Q)                                                                   \
+  while (mask[Q]) {                                                                       \
+    const int u = __ffs(mask[Q]) - 1;                                                     \
+    mask[Q] &= mask[Q] - 1u;                                                              \
+    q.template insert_fast<Q>(tile[t + kThreads * u],                                     \
+                              base + static_cast<uint32_t>(kThreads * u) - (Q));          \
+  }
+  TK_SURVIVORS(0)
+  TK_SURVIVORS(1)
+  TK_SURVIVORS(2)
+  TK_SURVIVORS(3)
+#undef TK_SURVIVORS
+}
+
+// Register queues per CTA of the TMA kernel: four per thread (float4 layout)
+// for k_b <= 2, max(256, b) for the sparse k_b > 2 layout.
+__host__ __device__ __forceinline__ int select_lanes(int kb, int b) {
+  return kb <= 2 ? kLanes : (b > kThreads ? b : kThreads);
+}
 
 constexpr int kConsumerWarps = kThreads / 32;
 constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
@@ -56,7 +131,7 @@ template <int KB>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs p, int stages,
                                                                   int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const SelectSmem L{stages, KB, cand_cap};
+  const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b)};
   float* ring = reinterpret_cast<float*>(smem);
   uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
@@ -120,6 +195,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
   }
 
   // ---------------- consumers
+  // k_b <= 2: four queues per thread over float4 positions (kLanes lanes),
+  // updated branch-free.  k_b > 2: queue q of thread t covers positions
+  // t + 256 q modulo nl = max(256, b) (select_tile_sparse), so each queue sees
+  // four times more elements and only the survivors of a threshold test pay
+  // for the sorted insert.
+  const int nl = select_lanes(KB, p.b);
+  const int nq = nl / kThreads;
   Queues<KB> q;
   int st = 0;       // ring stage of the next tile
   uint32_t ph = 0;  // its full-barrier parity
@@ -138,26 +220,31 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
       const bool ok = __any_sync(0xffffffffu,
                                  !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
-        const float* tile = ring + static_cast<size_t>(st) * kTile + 4 * tid;
-        const uint32_t pos0 = pos_thread + done;
-        constexpr int U = kTile / kLanes;
-        if (c == static_cast<uint32_t>(kTile)) {
-          float4 x[U];
-          uint32_t base[U];
+        if (KB <= 2) {
+          const float* tile = ring + static_cast<size_t>(st) * kTile + 4 * tid;
+          const uint32_t pos0 = pos_thread + done;
+          constexpr int U = kTile / kLanes;
+          if (c == static_cast<uint32_t>(kTile)) {
+            float4 x[U];
+            uint32_t base[U];
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            x[u] = *reinterpret_cast<const float4*>(tile + kLanes * u);
-            base[u] = pos0 + static_cast<uint32_t>(kLanes * u);
+            for (int u = 0; u < U; ++u) {
+              x[u] = *reinterpret_cast<const float4*>(tile + kLanes * u);
+              base[u] = pos0 + static_cast<uint32_t>(kLanes * u);
+            }
+            q.template offer_tile<U>(x, base);
+          } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const uint32_t off = 4u * tid + static_cast<uint32_t>(kLanes * u);
+              if (off < c)
+                q.offer4(*reinterpret_cast<const float4*>(tile + kLanes * u),
+                         pos0 + static_cast<uint32_t>(kLanes * u));
+            }
           }
-          q.template offer_tile<U>(x, base);
         } else {
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const uint32_t off = 4u * tid + static_cast<uint32_t>(kLanes * u);
-            if (off < c)
-              q.offer4(*reinterpret_cast<const float4*>(tile + kLanes * u),
-                       pos0 + static_cast<uint32_t>(kLanes * u));
-          }
+          select_tile_sparse<KB>(q, ring + static_cast<size_t>(st) * kTile, c,
+                                 static_cast<uint32_t>(a) + done, nq);
         }
       }
       __syncwarp();
@@ -170,11 +257,17 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
     }
     g = pend;
     // Piece done: publish the queues and finish (Stage 2 or cross-CTA merge).
+    if (KB <= 2) {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
+      for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
+    } else {
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        if (v < nq) q.store(v, lanebuf + static_cast<size_t>(tid + kThreads * v) * KB);
+    }
     group_sync(kThreads);
     finish_piece<KB, kGatherInput>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
-                                   p.x + row0, p.out_vals, p.out_idx, piece_flag);
+                                   p.x + row0, p.out_vals, p.out_idx, piece_flag, nl);
     group_sync(kThreads);
   }
 }
@@ -182,7 +275,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
 template <int KB>
 __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const SelectSmem L{0, KB, cand_cap};
+  const SelectSmem L{0, KB, cand_cap, kLanes};
   uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem);
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.lane_bytes());
   __shared__ int piece_flag;

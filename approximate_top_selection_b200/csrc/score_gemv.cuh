@@ -49,7 +49,9 @@ struct ScoreSmem {
   __host__ __device__ size_t shared_region() const {
     return sbuf_bytes() > lane_bytes() ? sbuf_bytes() : lane_bytes();
   }
-  __host__ __device__ size_t cand_bytes() const { return static_cast<size_t>(cand_cap) * 8; }
+  __host__ __device__ size_t cand_bytes() const {
+    return static_cast<size_t>(cand_cap) * 8 + kStage2Extra;
+  }
   __host__ __device__ size_t bar_bytes() const { return 16 * static_cast<size_t>(stages) + 16; }
   __host__ __device__ size_t total() const {
     return ring_bytes() + shared_region() + cand_bytes() + bar_bytes();

@@ -175,14 +175,14 @@ __device__ __forceinline__ void keep_best(uint64_t (&best)[KB], uint64_t c) {
   }
 }
 
-// Lane slot l (0 <= l < kLanes) holds the top-KB of the piece positions
-// congruent to l modulo L*b, with L = kLanes / b lanes per bucket (b <= kLanes),
+// Lane slot l (0 <= l < nl) holds the top-KB of the piece positions
+// congruent to l modulo L*b, with L = nl / b lanes per bucket (b <= nl),
 // so its bucket is (a + l) mod b for a piece starting at row position a.
 // Writes dst[j*KB + s], j = absolute bucket.  dst may be shared or global.
 template <int KB>
 __device__ __forceinline__ void merge_lanes(const uint64_t* lanebuf, int b, int64_t a,
-                                            uint64_t* dst, int T) {
-  const int L = kLanes / b;
+                                            uint64_t* dst, int T, int nl = kLanes) {
+  const int L = nl / b;
   const int a_mod = static_cast<int>(a % b);
   for (int beta = threadIdx.x; beta < b; beta += T) {
     uint64_t best[KB];
@@ -338,6 +338,119 @@ __host__ __device__ __forceinline__ int sort_capacity(int C) {
   return n;
 }
 
+// Shared-memory bytes of the Stage-2 buffer for C candidates: the sort
+// buffer plus the radix-select histogram and counters behind it.
+constexpr int kStage2Extra = 2048;
+__host__ __device__ __forceinline__ size_t stage2_bytes(int C) {
+  return static_cast<size_t>(sort_capacity(C)) * 8 + kStage2Extra;
+}
+
+template <ValueSource VS>
+__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const float* xrow,
+                                                  float* ov, int32_t* oi);
+
+// Stage 2 when the candidates far outnumber k: find the k-th largest packed
+// key with 8-bit radix histograms (most significant digit first; keys are
+// unique, so at most 8 passes, and the walk stops as soon as the boundary
+// digit holds exactly the elements still needed), gather the selected keys
+// and sort only those.  Same result as sorting all C and keeping k.
+template <int EPT, int VS>
+__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const float* xrow,
+                                                 float* ov, int32_t* oi) {
+  const int t = threadIdx.x;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(cand + sort_capacity(C));  // 256 bins
+  int* misc = reinterpret_cast<int*>(hist + 256);                        // digit, above, count, n
+  uint64_t v[EPT];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = t * EPT + j;
+    v[j] = e < C ? cand[e] : 0ull;
+  }
+  uint64_t prefix = 0;
+  int need = k;
+  int shift = 56;
+  bool all_real = false;
+  for (; shift >= 0; shift -= 8) {
+    for (int i = t; i < 256; i += kThreads) hist[i] = 0u;
+    group_sync(kThreads);
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const bool match = v[j] != 0ull && (shift == 56 || (v[j] >> (shift + 8)) == (prefix >> (shift + 8)));
+      // Candidates are often concentrated in a few bins: one atomic per
+      // distinct bin of the warp instead of one per lane.
+      const uint32_t bin = match ? static_cast<uint32_t>((v[j] >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (match && (t & 31) == __ffs(peers) - 1) atomicAdd(hist + bin, static_cast<uint32_t>(__popc(peers)));
+    }
+    group_sync(kThreads);
+    if (t < 32) {
+      // Lane l holds bins 255-8l down to 248-8l; find the digit that holds the
+      // need-th largest key.
+      int c8[8];
+      int local = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c8[i] = static_cast<int>(hist[255 - 8 * t - i]);
+        local += c8[i];
+      }
+      int incl = local;
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, m);
+        if (t >= m) incl += y;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+      if (t == 0) misc[3] = total;
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        if (t == l) {
+          int above = incl - local;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (above + c8[i] >= need) {
+              misc[0] = 255 - 8 * t - i;
+              misc[1] = above;
+              misc[2] = c8[i];
+              break;
+            }
+            above += c8[i];
+          }
+        }
+      }
+    }
+    group_sync(kThreads);
+    if (misc[3] < need) {  // fewer candidates than still needed: take them all
+      all_real = true;
+      group_sync(kThreads);
+      break;
+    }
+    const int d = misc[0], above = misc[1], cnt = misc[2];
+    group_sync(kThreads);  // misc is rewritten by the next pass
+    prefix |= static_cast<uint64_t>(d) << shift;
+    need -= above;
+    if (cnt == need) break;  // every key on this prefix is selected
+  }
+  // Selected: keys whose digits down to `shift` are >= the prefix (or, when
+  // there were fewer than needed, every real key matching the prefix so far).
+  if (t == 0) misc[3] = 0;
+  group_sync(kThreads);
+  const int sh = shift < 0 ? 0 : shift;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    bool sel;
+    if (all_real)
+      sel = v[j] != 0ull && (sh == 56 ? true : (v[j] >> (sh + 8)) >= (prefix >> (sh + 8)));
+    else
+      sel = v[j] != 0ull && (v[j] >> sh) >= (prefix >> sh);
+    if (sel) cand[atomicAdd(misc + 3, 1)] = v[j];
+  }
+  group_sync(kThreads);
+  const int kept = misc[3];
+  group_sync(kThreads);
+  finalize_row_fast<static_cast<ValueSource>(VS)>(cand, kept, k, xrow, ov, oi);
+}
+
 template <ValueSource VS>
 __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const float* xrow,
                                              float* ov, int32_t* oi, int T);
@@ -345,6 +458,10 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
 // Stage 2 for the streaming kernels (kThreads threads): up to 8 keys per
 // thread are sorted in registers; larger candidate sets use the shared-memory
 // network.
+template <int EPT, int VS>
+__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const float* xrow,
+                                                 float* ov, int32_t* oi);
+
 template <ValueSource VS>
 __device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const float* xrow,
                                                   float* ov, int32_t* oi) {
@@ -388,6 +505,21 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
   group_sync(T);
 }
 
+// Stage 2 entry of the streaming kernels: select first when that shrinks the
+// sort (at least 1024 candidates and k under half of them), else sort all.
+template <ValueSource VS>
+__device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const float* xrow, float* ov,
+                                       int32_t* oi) {
+  if (C >= 1024 && 2 * k <= C && C <= 16 * kThreads) {
+    switch (sort_capacity(C) / kThreads) {
+      case 4: finalize_row_select<4, VS>(cand, C, k, xrow, ov, oi); return;
+      case 8: finalize_row_select<8, VS>(cand, C, k, xrow, ov, oi); return;
+      default: finalize_row_select<16, VS>(cand, C, k, xrow, ov, oi); return;
+    }
+  }
+  finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
+}
+
 // ------------------------------------------------------------------ pieces
 struct RowSplit {
   int64_t rows, n;  // row length in elements (scores or keys)
@@ -409,22 +541,22 @@ __device__ __forceinline__ int64_t cta_start(const RowSplit& rs, int c) {
 template <int KB, ValueSource VS>
 __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_t a, int64_t len,
                              const uint64_t* lanebuf, uint64_t* cand, const float* xrow,
-                             float* out_vals, int32_t* out_idx, int* s_flag) {
+                             float* out_vals, int32_t* out_idx, int* s_flag, int nl = kLanes) {
   constexpr int T = kThreads;
   const int C = b * KB;
   float* ov = out_vals + r * static_cast<int64_t>(k);
   int32_t* oi = out_idx + r * static_cast<int64_t>(k);
   if (a == 0 && len == rs.n) {
-    merge_lanes<KB>(lanebuf, b, 0, cand, T);
+    merge_lanes<KB>(lanebuf, b, 0, cand, T, nl);
     group_sync(T);
-    finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
+    stage2<VS>(cand, C, k, xrow, ov, oi);
     return;
   }
   const int64_t row0 = r * rs.n;
   const int me = blockIdx.x;
   const int slot = (cta_start(rs, me) / rs.n == r) ? 0 : 1;
   uint64_t* mine = rs.slots + (static_cast<size_t>(me) * 2 + slot) * C;
-  merge_lanes<KB>(lanebuf, b, a, mine, T);
+  merge_lanes<KB>(lanebuf, b, a, mine, T, nl);
   __threadfence();
   group_sync(T);
   const int c_first = part_of(row0, rs.units, rs.G, rs.align);
@@ -456,7 +588,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
     for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
   }
   group_sync(T);
-  finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
+  stage2<VS>(cand, C, k, xrow, ov, oi);
   if (threadIdx.x == 0) rs.tickets[r] = 0u;  // leave the workspace zeroed
 }
 

@@ -194,16 +194,16 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
   const int C = b * KB;
   pl->cand_cap = sort_capacity(C);
   pl->align = fast ? 4 : 1;
-  pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap}, 2) : 0;
+  pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap, select_lanes(KB, b)}, 2) : 0;
   int per_sm = 0;
   if (fast) {
-    SelectSmem L{pl->stages, KB, pl->cand_cap};
+    SelectSmem L{pl->stages, KB, pl->cand_cap, select_lanes(KB, b)};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
     int rc = occupancy(bucket_select_tma<KB>, kPipeThreads, pl->smem, &per_sm);
     if (rc) return rc;
   } else {
-    SelectSmem L{0, KB, pl->cand_cap};
+    SelectSmem L{0, KB, pl->cand_cap, kLanes};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
     int rc = occupancy(bucket_select_general<KB>, kThreads, pl->smem, &per_sm);
@@ -413,7 +413,7 @@ int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n
   clear_launch_error();
   score_select_umma<KB, D><<<grid, kUmmaThreads, smem, st>>>(tmQ, tmK, a);
   if ((rc = launch_status())) return rc;
-  const size_t fsmem = static_cast<size_t>(sort_capacity(b * KB)) * 8;
+  const size_t fsmem = stage2_bytes(b * KB);
   umma_finish<KB><<<static_cast<unsigned>(rows), kThreads, fsmem, st>>>(
       a.cand, rows, b, k, out_vals, out_idx);
   return launch_status();
