@@ -157,6 +157,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait_then_release();
 
   // Tile t of this CTA covers [g, g + len) with len = min(kTile, e0 - g,
   // end of g's row - g): tiles never straddle rows.
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, 
   const int64_t n = rs.n;
   const int b = p.b;
   const int W = (kLanes / b) * b;  // stripe: lanes per bucket times b
+  pdl_wait_then_release();
 
   Queues<KB> q;
   int64_t g = s0;

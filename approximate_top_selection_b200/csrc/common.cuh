@@ -51,6 +51,16 @@ __device__ __forceinline__ float fmin_nan(float a, float b) {
   return d;
 }
 
+// Programmatic dependent launch.  Kernels are launched so that they may start
+// while the previous kernel of the stream finishes; every thread waits here
+// (until that kernel has completed and its writes are visible) before it
+// touches global memory, and then lets the next kernel of the stream start
+// its own set-up early in the same way.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier / bulk copy
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

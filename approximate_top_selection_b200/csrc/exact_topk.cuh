@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(kExactThreads) exact_topk_kernel(const float* 
   int32_t* oi = out_idx + r * static_cast<int64_t>(k);
   const int tid = threadIdx.x;
   const int T = blockDim.x;
+  pdl_wait_then_release();
 
   if (n <= kSortCap) {
     uint64_t* s = reinterpret_cast<uint64_t*>(smem);

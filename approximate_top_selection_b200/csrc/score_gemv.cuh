@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kScorePipeThreads, 2)
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait_then_release();
 
   if (warp == kScoreConsumerWarps) {  // ---------------- producer
     if (lane == 0) {

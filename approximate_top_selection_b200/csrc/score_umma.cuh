@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait_then_release();
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -440,6 +441,7 @@ __global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem);
   const int64_t r = blockIdx.x;
+  pdl_wait_then_release();
   for (int j = threadIdx.x; j < b; j += kThreads) {
     uint64_t best[KB];
 #pragma unroll

@@ -308,21 +308,43 @@ int launch_status() {
   return e == cudaSuccess ? TOPK_OK : TOPK_ECUDA;
 }
 
+// Launch with programmatic stream serialisation: the kernel may begin while
+// the previous kernel on the stream finishes; it waits on the device
+// (griddepcontrol.wait) before reading or writing global memory.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  clear_launch_error();
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return TOPK_ECUDA;
+  }
+  return launch_status();
+}
+
 template <int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs& a, cudaStream_t st) {
-  clear_launch_error();
   if (fast)
-    bucket_select_tma<KB><<<pl.G, kPipeThreads, pl.smem, st>>>(a, pl.stages, pl.cand_cap);
-  else
-    bucket_select_general<KB><<<pl.G, kThreads, pl.smem, st>>>(a, pl.cand_cap);
-  return launch_status();
+    return launch_pdl(bucket_select_tma<KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
+                      pl.stages, pl.cand_cap);
+  return launch_pdl(bucket_select_general<KB>, dim3(pl.G), dim3(kThreads), pl.smem, st, a,
+                    pl.cand_cap);
 }
 
 template <int KB, int D>
 int launch_score_kd(const Plan& pl, const ScoreArgs& a, cudaStream_t st) {
-  clear_launch_error();
-  score_select_gemv<KB, D><<<pl.G, kScorePipeThreads, pl.smem, st>>>(a, pl.stages, pl.cand_cap);
-  return launch_status();
+  return launch_pdl(score_select_gemv<KB, D>, dim3(pl.G), dim3(kScorePipeThreads), pl.smem, st, a,
+                    pl.stages, pl.cand_cap);
 }
 
 template <int KB>
@@ -410,13 +432,12 @@ int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n
   if ((rc = prepare_kernel(score_select_umma<KB, D>))) return rc;
   if ((rc = prepare_kernel(umma_finish<KB>))) return rc;
   const int grid = std::min(a.units, dev.sms);
-  clear_launch_error();
-  score_select_umma<KB, D><<<grid, kUmmaThreads, smem, st>>>(tmQ, tmK, a);
-  if ((rc = launch_status())) return rc;
+  if ((rc = launch_pdl(score_select_umma<KB, D>, dim3(grid), dim3(kUmmaThreads), smem, st, tmQ, tmK,
+                       a)))
+    return rc;
   const size_t fsmem = stage2_bytes(b * KB);
-  umma_finish<KB><<<static_cast<unsigned>(rows), kThreads, fsmem, st>>>(
-      a.cand, rows, b, k, out_vals, out_idx);
-  return launch_status();
+  return launch_pdl(umma_finish<KB>, dim3(static_cast<unsigned>(rows)), dim3(kThreads), fsmem, st,
+                    a.cand, rows, b, k, out_vals, out_idx);
 }
 
 template <int KB>
@@ -581,11 +602,8 @@ int topk_exact(const float* scores, int64_t rows, int64_t n, int k, float* out_v
   const size_t smem = L.total();
   if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
   if ((rc = prepare_kernel(exact_topk_kernel))) return rc;
-  clear_launch_error();
-  exact_topk_kernel<<<static_cast<unsigned>(rows), kExactThreads, smem,
-                      static_cast<cudaStream_t>(stream)>>>(scores, n, k, L.sel_cap, out_vals,
-                                                           out_idx);
-  return launch_status();
+  return launch_pdl(exact_topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(kExactThreads), smem,
+                    static_cast<cudaStream_t>(stream), scores, n, k, L.sel_cap, out_vals, out_idx);
 }
 
 int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,
