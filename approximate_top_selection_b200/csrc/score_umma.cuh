@@ -9,18 +9,19 @@
 //
 // Work unit = (128 queries, group of 8 buckets).  Entity e = t*b + j belongs to
 // bucket j, so a unit walks the entities t*b + 8g + jj (jj < 8) for all t.  The
-// TMA engine fetches them as a 3-D box {64 d, 8 jj, 32 t} of the key matrix
-// viewed as [T][b][d]: 256 key rows of 128 B with the 128-byte swizzle, which is
-// exactly a K-major UMMA B operand.  Accumulator column c of a 128 x 256 tile
-// is then entity (t0 + c/8)*b + 8g + c%8, i.e. bucket 8g + c%8, and each
-// epilogue thread (one query row) keeps only 8 bucket queues in registers.
+// TMA engine fetches, per bucket jj, the box {64 d, 1, 32 t} of the key matrix
+// viewed as [T][b][d], one after the other: 256 key rows of 128 B with the
+// 128-byte swizzle, bucket-major -- exactly a K-major UMMA B operand.
+// Accumulator column c of a 128 x 256 tile is then entity
+// (t0 + c%32)*b + 8g + c/32: each 32-column TMEM load is one bucket's 32
+// stripes, so an epilogue warp owns whole buckets and needs no merge.
 //
 // Warp roles (320 threads): warp 0 issues TMA loads (Q tile once per unit, key
 // stages through a ring), warp 1 owns TMEM (512 columns = two 128x256 fp32
 // accumulators) and issues the MMAs from one thread, warps 2..9 drain TMEM
-// (tcgen05.ld) and update the queues: two warps per TMEM lane quarter, one per
-// half of the 256 columns.  Per-unit results (top-k_b per bucket and column half)
-// go to the workspace; umma_finish merges the halves and runs Stage 2.
+// (tcgen05.ld) and update the queues: H warps per TMEM lane quarter, each
+// owning 8/H buckets (H = 4 for k_b <= 2, 2 for larger queues).  Per-unit
+// results (top-k_b per bucket) go to the workspace; umma_finish runs Stage 2.
 //
 // The units of one bucket group are consecutive, so the 8 query tiles that read
 // the same key rows run at about the same time and share them through L2.
@@ -38,16 +39,20 @@ constexpr int kUmmaGroup = 8;          // buckets per unit
 constexpr int kUmmaTPerTile = kUmmaN / kUmmaGroup;  // 32 stripes per tile
 constexpr int kUmmaChunkBytes = 16384;              // 128 rows x 64 bf16 (A chunk)
 constexpr int kUmmaStageBytes = 32768;              // 256 rows x 64 bf16 (B stage)
-constexpr int kUmmaStages = 4;
-constexpr int kUmmaThreads = 320;
-constexpr int kUmmaEpiWarps = 8;
+#ifndef TOPK_UMMA_STAGES
+#define TOPK_UMMA_STAGES 4
+#endif
+constexpr int kUmmaStages = TOPK_UMMA_STAGES;
+// Epilogue warps: 8 (k_b > 2, more registers per thread) or 16 (k_b <= 2).
+__host__ __device__ constexpr int umma_epi_warps(int kb) { return kb <= 2 ? 16 : 8; }
+__host__ __device__ constexpr int umma_threads(int kb) { return 64 + 32 * umma_epi_warps(kb); }
 
 struct UmmaArgs {
   int64_t rows, n;   // queries, entities
   int b, T;          // buckets, stripes (n = T * b)
   int mtiles, groups, tiles_per_unit, units;
   float* out_scores;  // nullable [rows][n]
-  uint64_t* cand;     // [rows][b][2][KB]
+  uint64_t* cand;     // [rows][b][KB]
 };
 
 template <int D>
@@ -186,51 +191,62 @@ struct BucketQueues {
   }
 };
 
-// Feeds the 32 scores of one tcgen05.ld (columns c0 .. c0+31 of the tile, c0 a
-// multiple of 32, so column r belongs to queue r % 8 and stripe c0/8 + r/8).
-template <int KB>
-__device__ __forceinline__ void umma_feed(BucketQueues<kUmmaGroup, KB>& q, const uint32_t (&r)[32],
-                                          int c0, int t0, int T, uint32_t b, uint32_t jbase,
-                                          int64_t row, int64_t rows, int64_t n, float* out_scores) {
+// Feeds the 32 scores of one tcgen05.ld -- bucket jb's stripes t0 .. t0+31 --
+// to queue QI (a runtime index unrolled by the caller).  Queues store the
+// stripe t; the entity t*b + jb is formed when the queue is written out.
+template <int KB, int NQ, int QI>
+__device__ __forceinline__ void umma_feed_bucket(BucketQueues<NQ, KB>& q, const uint32_t (&r)[32],
+                                                 int t0, int T, uint32_t b, uint32_t jb, int64_t row,
+                                                 int64_t rows, int64_t n, float* out_scores) {
   float m = __uint_as_float(r[0]);
 #pragma unroll
   for (int i = 1; i < 32; ++i) m = fmin_nan(m, __uint_as_float(r[i]));
   const bool special = !(m > __int_as_float(0xff800000));
-  const int tfirst = t0 + c0 / kUmmaGroup;
-  const bool full = tfirst + 4 <= T;
+  const int valid = T - t0 < 32 ? T - t0 : 32;  // stripes of this tile inside the tensor
   if (out_scores != nullptr && row < rows) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int t = tfirst + i / kUmmaGroup;
-      if (t < T)
-        out_scores[row * n + static_cast<int64_t>(t) * b + jbase + (i % kUmmaGroup)] =
-            __uint_as_float(r[i]);
-    }
+    for (int i = 0; i < 32; ++i)
+      if (i < valid)
+        out_scores[row * n + static_cast<int64_t>(t0 + i) * b + jb] = __uint_as_float(r[i]);
   }
-#define TK_FEED_ONE(I)                                                                    \
-  {                                                                                       \
-    const int t = tfirst + (I) / kUmmaGroup;                                              \
-    const uint32_t e = static_cast<uint32_t>(t) * b + jbase + ((I) % kUmmaGroup);          \
-    if (full || t < T) {                                                                  \
-      if (special)                                                                        \
-        q.template insert_exact<(I) % kUmmaGroup>(__uint_as_float(r[I]), e);              \
-      else                                                                                \
-        q.template insert_fast<(I) % kUmmaGroup>(__uint_as_float(r[I]), e);               \
-    }                                                                                     \
+  if (!special && valid == 32) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      q.template insert_fast<QI>(__uint_as_float(r[i]), static_cast<uint32_t>(t0 + i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid) q.template insert_exact<QI>(__uint_as_float(r[i]), static_cast<uint32_t>(t0 + i));
   }
-  TK_FEED_ONE(0) TK_FEED_ONE(1) TK_FEED_ONE(2) TK_FEED_ONE(3) TK_FEED_ONE(4) TK_FEED_ONE(5)
-  TK_FEED_ONE(6) TK_FEED_ONE(7) TK_FEED_ONE(8) TK_FEED_ONE(9) TK_FEED_ONE(10) TK_FEED_ONE(11)
-  TK_FEED_ONE(12) TK_FEED_ONE(13) TK_FEED_ONE(14) TK_FEED_ONE(15) TK_FEED_ONE(16)
-  TK_FEED_ONE(17) TK_FEED_ONE(18) TK_FEED_ONE(19) TK_FEED_ONE(20) TK_FEED_ONE(21)
-  TK_FEED_ONE(22) TK_FEED_ONE(23) TK_FEED_ONE(24) TK_FEED_ONE(25) TK_FEED_ONE(26)
-  TK_FEED_ONE(27) TK_FEED_ONE(28) TK_FEED_ONE(29) TK_FEED_ONE(30) TK_FEED_ONE(31)
-#undef TK_FEED_ONE
+}
+
+// All NQ buckets of a warp, one 32-column TMEM load at a time (queue index
+// fixed at compile time).  After the last load the accumulator buffer is
+// handed back to the MMA warp before the last bucket is processed.
+template <int KB, int NQ, int J>
+__device__ __forceinline__ void umma_feed_all(BucketQueues<NQ, KB>& q, uint32_t taddr,
+                                              uint64_t* acc_empty_buf, int t0, int T, uint32_t b,
+                                              uint32_t jbase, int64_t row, int64_t rows, int64_t n,
+                                              float* out_scores) {
+  uint32_t r[32];
+  tmem_ld_x32(taddr + J * 32, r);
+  if constexpr (J + 1 == NQ) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(acc_empty_buf);
+  }
+  umma_feed_bucket<KB, NQ, J>(q, r, t0, T, b, jbase + J, row, rows, n, out_scores);
+  if constexpr (J + 1 < NQ)
+    umma_feed_all<KB, NQ, J + 1>(q, taddr, acc_empty_buf, t0, T, b, jbase, row, rows, n, out_scores);
 }
 
 template <int KB, int D>
-__global__ void __launch_bounds__(kUmmaThreads, 1)
+__global__ void __launch_bounds__(umma_threads(KB), 1)
     score_select_umma(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       UmmaArgs p) {
+  constexpr int kEpiWarps = umma_epi_warps(KB);
+  constexpr int H = kEpiWarps / 4;             // warps sharing one TMEM lane quarter
+  constexpr int kColsPerWarp = kUmmaN / H;     // accumulator columns each of them drains
   using L = UmmaSmem<D>;
   constexpr int kChunks = L::kChunks;
   constexpr uint32_t kIdesc = umma_idesc_bf16(kUmmaM, kUmmaN);
@@ -261,7 +277,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(acc_full + s, 1);
-      mbar_init(acc_empty + s, kUmmaEpiWarps);
+      mbar_init(acc_empty + s, kEpiWarps);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -302,8 +318,10 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
               break;
             }
             mbar_expect_tx(full_b + st, kUmmaStageBytes);
-            tma_load_3d(b_ring + st * kUmmaStageBytes, &tmK, c * 64, g * kUmmaGroup,
-                        tile * kUmmaTPerTile, full_b + st);
+#pragma unroll
+            for (int jj = 0; jj < kUmmaGroup; ++jj)
+              tma_load_3d(b_ring + st * kUmmaStageBytes + jj * (kUmmaStageBytes / kUmmaGroup), &tmK,
+                          c * 64, g * kUmmaGroup + jj, tile * kUmmaTPerTile, full_b + st);
             ++bt;
             if (++st == kUmmaStages) {
               st = 0;
@@ -374,14 +392,15 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - 2;
     const int quarter = warp & 3;            // TMEM lanes this warp may read
-    const int half = ew >> 2;                // which 128 columns of the tile
+    const int slice = ew >> 2;               // which buckets of the group (0 .. H-1)
+    constexpr int kBucketsPerWarp = kUmmaGroup / H;
     const int64_t row_in_tile = quarter * 32 + lane;
-    BucketQueues<kUmmaGroup, KB> q;
+    BucketQueues<kBucketsPerWarp, KB> q;
     int64_t tg = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
       const int m = u % p.mtiles, g = u / p.mtiles;
       const int64_t row = static_cast<int64_t>(m) * kUmmaM + row_in_tile;
-      const uint32_t jbase = static_cast<uint32_t>(g * kUmmaGroup);
+      const uint32_t jbase = static_cast<uint32_t>(g * kUmmaGroup + slice * kBucketsPerWarp);
       q.reset();
       bool ok = true;
       for (int tile = 0; tile < p.tiles_per_unit; ++tile, ++tg) {
@@ -393,33 +412,23 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int t0 = tile * kUmmaTPerTile;
-        const uint32_t taddr =
-            tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(buf * kUmmaN);
-#pragma unroll 1
-        for (int i = 0; i < 4; ++i) {
-          const int c0 = half * 128 + i * 32;
-          uint32_t r[32];
-          tmem_ld_x32(taddr + static_cast<uint32_t>(c0), r);
-          if (i == 3) {
-            // Everything of this buffer is in registers: hand it back to the MMA.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty + buf);
-          }
-          umma_feed<KB>(q, r, c0, t0, p.T, static_cast<uint32_t>(p.b), jbase, row, p.rows, p.n,
-                        p.out_scores);
-        }
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(buf * kUmmaN + slice * kBucketsPerWarp * 32);
+        umma_feed_all<KB, kBucketsPerWarp, 0>(q, taddr, acc_empty + buf, t0, p.T,
+                                              static_cast<uint32_t>(p.b), jbase, row, p.rows, p.n,
+                                              p.out_scores);
       }
       if (!ok) break;
       if (row < p.rows) {
-        uint64_t* dst = p.cand + ((static_cast<size_t>(row) * p.b + jbase) * 2 + half) * KB;
+        uint64_t* dst = p.cand + (static_cast<size_t>(row) * p.b + jbase) * KB;
 #pragma unroll
-        for (int j = 0; j < kUmmaGroup; ++j)
+        for (int jj = 0; jj < kBucketsPerWarp; ++jj)
 #pragma unroll
-          for (int s = 0; s < KB; ++s)
-            dst[static_cast<size_t>(j) * 2 * KB + s] =
-                q.idx[j][s] != BucketQueues<kUmmaGroup, KB>::kEmpty
-                    ? pack(order_key(q.val[j][s]), q.idx[j][s])
+          for (int s2 = 0; s2 < KB; ++s2)
+            dst[static_cast<size_t>(jj) * KB + s2] =
+                q.idx[jj][s2] != BucketQueues<kBucketsPerWarp, KB>::kEmpty
+                    ? pack(order_key(q.val[jj][s2]),
+                           q.idx[jj][s2] * static_cast<uint32_t>(p.b) + jbase + jj)
                     : 0ull;
       }
     }
@@ -433,11 +442,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1)
   }
 }
 
-// Stage 2 of the tensor-core path: per query, the top-k_b of each bucket over
-// the two column halves, then the exact top-k of the b*k_b candidates.
+// Stage 2 of the tensor-core path: per query, the exact top-k of the b*k_b
+// bucket candidates (the workspace is cleared behind the reads).
 template <int KB>
 __global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64_t rows, int b,
                                                         int k, float* out_vals, int32_t* out_idx) {
+
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem);
   const int64_t r = blockIdx.x;
@@ -446,9 +456,9 @@ __global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64
     uint64_t best[KB];
 #pragma unroll
     for (int s = 0; s < KB; ++s) best[s] = 0;
-    uint64_t* src = cand_ws + (static_cast<size_t>(r) * b + j) * 2 * KB;
+    uint64_t* src = cand_ws + (static_cast<size_t>(r) * b + j) * KB;
 #pragma unroll
-    for (int s = 0; s < 2 * KB; ++s) {
+    for (int s = 0; s < KB; ++s) {
       keep_best<KB>(best, src[s]);
       src[s] = 0ull;  // leave the workspace zeroed for the next call
     }

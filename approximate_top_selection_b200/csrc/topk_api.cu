@@ -364,7 +364,7 @@ bool umma_eligible(int64_t rows, int64_t n, int64_t kstride, int b, int d) {
 }
 
 size_t umma_workspace(int64_t rows, int b, int kb) {
-  return static_cast<size_t>(rows) * b * 2 * kb * 8;
+  return static_cast<size_t>(rows) * b * kb * 8;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -409,7 +409,7 @@ int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n
                                 static_cast<cuuint64_t>(T)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                                    static_cast<cuuint64_t>(b) * D * 2};
-    const cuuint32_t box[3] = {64, kUmmaGroup, kUmmaTPerTile};
+    const cuuint32_t box[3] = {64, 1, kUmmaTPerTile};  // one bucket's 32 stripes per load
     const cuuint32_t es[3] = {1, 1, 1};
     if (encode(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(K), dims, strides,
                box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -432,8 +432,8 @@ int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n
   if ((rc = prepare_kernel(score_select_umma<KB, D>))) return rc;
   if ((rc = prepare_kernel(umma_finish<KB>))) return rc;
   const int grid = std::min(a.units, dev.sms);
-  if ((rc = launch_pdl(score_select_umma<KB, D>, dim3(grid), dim3(kUmmaThreads), smem, st, tmQ, tmK,
-                       a)))
+  if ((rc = launch_pdl(score_select_umma<KB, D>, dim3(grid), dim3(umma_threads(KB)), smem, st, tmQ,
+                       tmK, a)))
     return rc;
   const size_t fsmem = stage2_bytes(b * KB);
   return launch_pdl(umma_finish<KB>, dim3(static_cast<unsigned>(rows)), dim3(kThreads), fsmem, st,
