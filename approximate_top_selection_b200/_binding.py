@@ -16,7 +16,7 @@ import torch
 from . import build as _build
 
 TOPK_OK, TOPK_EINVAL, TOPK_EUNSUPPORTED, TOPK_ECUDA, TOPK_EWORKSPACE, TOPK_ESCRATCH = range(6)
-TOPK_OP_BUCKETED, TOPK_OP_EXACT, TOPK_OP_SCORE = range(3)
+TOPK_OP_BUCKETED, TOPK_OP_EXACT, TOPK_OP_SCORE, TOPK_OP_BUCKETED_BF16 = range(4)
 
 _lib = None
 _lock = threading.Lock()
@@ -54,6 +54,8 @@ def load_library():
             lib.topk_exact.restype = i32
             lib.score_topk.argtypes = [p, i64, i32, p, i64, i64, i32, i32, i32, p, p, p, p, sz, p]
             lib.score_topk.restype = i32
+            lib.topk_bucketed_bf16.argtypes = [p, i64, i64, i32, i32, i32, p, p, p, sz, p]
+            lib.topk_bucketed_bf16.restype = i32
             lib.topk_bucketed_noalloc.argtypes = [p, i64, i64, i32, i32, i32, p, p, p]
             lib.topk_bucketed_noalloc.restype = i32
             lib.topk_status_string.argtypes = [i32]
@@ -117,12 +119,12 @@ def topk_workspace_bytes(op: int, rows: int, n: int, k: int, b: int = 1, kb: int
     return v
 
 
-def _outputs(rows: int, k: int, device, out_vals, out_idx):
+def _outputs(rows: int, k: int, device, out_vals, out_idx, dtype=torch.float32):
     if out_vals is None:
-        out_vals = torch.empty(rows, k, dtype=torch.float32, device=device)
+        out_vals = torch.empty(rows, k, dtype=dtype, device=device)
     if out_idx is None:
         out_idx = torch.empty(rows, k, dtype=torch.int32, device=device)
-    _cuda(out_vals, "out_vals", torch.float32)
+    _cuda(out_vals, "out_vals", dtype)
     _cuda(out_idx, "out_idx", torch.int32)
     if out_vals.numel() != rows * k or out_idx.numel() != rows * k:
         raise ValueError("outputs must hold rows*k elements")
@@ -131,11 +133,15 @@ def _outputs(rows: int, k: int, device, out_vals, out_idx):
 
 def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=None, out_idx=None,
                   workspace: torch.Tensor | None = None, stream=None):
-    """Bucketed approximate top-k of every row of `scores` ([rows, n] float32, CUDA).
+    """Bucketed approximate top-k of every row of `scores` ([rows, n] float32
+    or bfloat16, CUDA).
 
-    Returns (values [rows, k] float32, indices [rows, k] int32), best-first,
-    padded with -inf / -1.
+    Returns (values [rows, k] of the input dtype, indices [rows, k] int32),
+    best-first, padded with -inf / -1.
     """
+    if isinstance(scores, torch.Tensor) and scores.dtype == torch.bfloat16:
+        return topk_bucketed_bf16(scores, k, b, kb, out_vals=out_vals, out_idx=out_idx,
+                                  workspace=workspace, stream=stream)
     lib = load_library()
     _cuda(scores, "scores", torch.float32)
     if scores.dim() != 2:
@@ -150,6 +156,26 @@ def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=Non
                                out_idx.data_ptr(), ws.data_ptr() if ws is not None else None,
                                ws.numel() if ws is not None else 0, sh)
     _check(st, "topk_bucketed")
+    return out_vals, out_idx
+
+
+def topk_bucketed_bf16(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=None,
+                       out_idx=None, workspace: torch.Tensor | None = None, stream=None):
+    """Bucketed approximate top-k of bfloat16 rows; values come back as bf16."""
+    lib = load_library()
+    _cuda(scores, "scores", torch.bfloat16)
+    if scores.dim() != 2:
+        raise ValueError("scores must be [rows, n]")
+    rows, n = scores.shape
+    with torch.cuda.device(scores.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx, torch.bfloat16)
+        need = topk_workspace_bytes(TOPK_OP_BUCKETED_BF16, rows, n, k, b, kb)
+        ws = workspace if workspace is not None else _workspace(need, scores.device, sh)
+        st = lib.topk_bucketed_bf16(scores.data_ptr(), rows, n, k, b, kb, out_vals.data_ptr(),
+                                    out_idx.data_ptr(), ws.data_ptr() if ws is not None else None,
+                                    ws.numel() if ws is not None else 0, sh)
+    _check(st, "topk_bucketed_bf16")
     return out_vals, out_idx
 
 

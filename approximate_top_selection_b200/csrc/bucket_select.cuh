@@ -23,12 +23,37 @@
 
 namespace tk {
 
-constexpr int kTile = 8192;  // floats per bulk copy (32 KB)
+constexpr int kTileBytes = 32768;  // bytes per bulk copy
+constexpr int kTile = 8192;        // fp32 elements per tile
 
+// Element types of score rows: float, or uint16_t holding bfloat16 bits.  A
+// bf16 widened to fp32 is exact and keeps the order, ties, -0 and NaN, so the
+// queues always compare fp32 values.
+template <typename T>
+struct Elem {
+  static constexpr int kPerTile = kTileBytes / static_cast<int>(sizeof(T));
+  static constexpr int kAlign = 16 / static_cast<int>(sizeof(T));  // elements per 16 bytes
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(uint16_t h) {
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+// Four consecutive elements (16 or 8 bytes, aligned) as fp32.
+__device__ __forceinline__ float4 load4_f32(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 load4_f32(const uint16_t* p) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                     __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+}
+
+template <typename T>
 struct SelectArgs {
-  const float* x;
+  const T* x;
   int k, b;
-  float* out_vals;
+  T* out_vals;
   int32_t* out_idx;
   RowSplit rs;
 };
@@ -36,7 +61,9 @@ struct SelectArgs {
 // Shared-memory layout of the selection kernels (bytes).
 struct SelectSmem {
   int stages, kb, cand_cap, nl;  // nl: register queues (lanes) per CTA
-  __host__ __device__ size_t ring_bytes() const { return static_cast<size_t>(stages) * kTile * 4; }
+  __host__ __device__ size_t ring_bytes() const {
+    return static_cast<size_t>(stages) * kTileBytes;
+  }
   __host__ __device__ size_t lane_bytes() const { return static_cast<size_t>(nl) * kb * 8; }
   __host__ __device__ size_t cand_bytes() const {
     return static_cast<size_t>(cand_cap) * 8 + kStage2Extra;
@@ -54,17 +81,17 @@ struct SelectSmem {
 // queues have filled -- go through the sorted insert, re-read from shared
 // memory, so a warp pays for its busiest thread's survivors rather than for
 // every element.  A tile holding NaN or -inf takes the exact update instead.
-template <int KB>
-__device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const float* tile, uint32_t c,
+template <int KB, typename T>
+__device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile, uint32_t c,
                                                    uint32_t pos_tile, int nq) {
-  constexpr int U = kTile / kThreads;  // 32 elements per thread
+  constexpr int U = kTile / kThreads;  // 32 elements per thread (8192 per call)
   const int t = threadIdx.x;
   float x[U];
   float m = __int_as_float(0x7f800000);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const bool valid = static_cast<uint32_t>(t + kThreads * u) < c;
-    x[u] = valid ? tile[t + kThreads * u] : __int_as_float(0x7f800000);
+    x[u] = valid ? to_f32(tile[t + kThreads * u]) : __int_as_float(0x7f800000);
     m = fmin_nan(m, x[u]);
   }
   const uint32_t base = pos_tile + static_cast<uint32_t>(t);
@@ -104,7 +131,7 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const float* t
   while (mask[Q]) {                                                                       \
     const int u = __ffs(mask[Q]) - 1;                                                     \
     mask[Q] &= mask[Q] - 1u;                                                              \
-    q.template insert_fast<Q>(tile[t + kThreads * u],                                     \
+    q.template insert_fast<Q>(to_f32(tile[t + kThreads * u]),                             \
                               base + static_cast<uint32_t>(kThreads * u) - (Q));          \
   }
   TK_SURVIVORS(0)
@@ -127,12 +154,13 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // the CTA's tiles into a ring of `stages` shared-memory stages (full barrier:
 // bytes landed; empty barrier: every consumer warp is done with the stage);
 // the kThreads consumer threads never wait for each other inside a piece.
-template <int KB>
-__global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs p, int stages,
+template <typename T, int KB>
+__global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
                                                                   int cand_cap) {
+  constexpr int kTileElems = Elem<T>::kPerTile;
   extern __shared__ __align__(128) unsigned char smem[];
   const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b)};
-  float* ring = reinterpret_cast<float*>(smem);
+  T* ring = reinterpret_cast<T*>(smem);
   uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
   uint64_t* full =
@@ -159,13 +187,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
   __syncthreads();
   pdl_wait_then_release();
 
-  // Tile t of this CTA covers [g, g + len) with len = min(kTile, e0 - g,
+  // Tile t of this CTA covers [g, g + len) with len = min(tile, e0 - g,
   // end of g's row - g): tiles never straddle rows.
   auto tile_len = [&](int64_t g) -> int64_t {
     const int64_t rowend = (g / n + 1) * n;
     int64_t c = e0 - g;
     if (rowend - g < c) c = rowend - g;
-    return c < kTile ? c : kTile;
+    return c < kTileElems ? c : kTileElems;
   };
 
   if (warp == kConsumerWarps) {  // ---------------- producer
@@ -176,9 +204,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
       while (g < e0) {
         const int64_t c = tile_len(g);
         if (t >= stages && !mbar_wait_or_abort(empty + st, ph ^ 1u, abort_flag)) break;
-        const uint32_t bytes = static_cast<uint32_t>(c * 4);
+        const uint32_t bytes = static_cast<uint32_t>(c * static_cast<int64_t>(sizeof(T)));
         mbar_expect_tx(full + st, bytes);
-        bulk_g2s(ring + static_cast<size_t>(st) * kTile, p.x + g, bytes, full + st);
+        bulk_g2s(ring + static_cast<size_t>(st) * kTileElems, p.x + g, bytes, full + st);
         g += c;
         ++t;
         if (++st == stages) {
@@ -196,7 +224,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
   }
 
   // ---------------- consumers
-  // k_b <= 2: four queues per thread over float4 positions (kLanes lanes),
+  // k_b <= 2: four queues per thread over 4-element groups (kLanes lanes),
   // updated branch-free.  k_b > 2: queue q of thread t covers positions
   // t + 256 q modulo nl = max(256, b) (select_tile_sparse), so each queue sees
   // four times more elements and only the survivors of a threshold test pay
@@ -216,36 +244,47 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
     const uint32_t pos_thread = static_cast<uint32_t>(a) + 4u * tid;
     q.reset();
     for (uint32_t done = 0; done < len;) {
-      const uint32_t c = (len - done) < static_cast<uint32_t>(kTile) ? (len - done) : kTile;
+      const uint32_t c =
+          (len - done) < static_cast<uint32_t>(kTileElems) ? (len - done) : kTileElems;
       // Warp-uniform: if any lane saw the stage complete, its bytes have landed.
       const bool ok = __any_sync(0xffffffffu,
                                  !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
+        const T* stage_tile = ring + static_cast<size_t>(st) * kTileElems;
         if (KB <= 2) {
-          const float* tile = ring + static_cast<size_t>(st) * kTile + 4 * tid;
-          const uint32_t pos0 = pos_thread + done;
+          // In slices of kTile elements (a bf16 tile holds two of them).
           constexpr int U = kTile / kLanes;
-          if (c == static_cast<uint32_t>(kTile)) {
-            float4 x[U];
-            uint32_t base[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-              x[u] = *reinterpret_cast<const float4*>(tile + kLanes * u);
-              base[u] = pos0 + static_cast<uint32_t>(kLanes * u);
-            }
-            q.template offer_tile<U>(x, base);
-          } else {
+          for (int h = 0; h < kTileElems / kTile; ++h) {
+            const uint32_t hoff = static_cast<uint32_t>(h * kTile);
+            const T* tile = stage_tile + hoff + 4 * tid;
+            const uint32_t pos0 = pos_thread + done + hoff;
+            if (hoff + kTile <= c) {
+              float4 x[U];
+              uint32_t base[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-              const uint32_t off = 4u * tid + static_cast<uint32_t>(kLanes * u);
-              if (off < c)
-                q.offer4(*reinterpret_cast<const float4*>(tile + kLanes * u),
-                         pos0 + static_cast<uint32_t>(kLanes * u));
+              for (int u = 0; u < U; ++u) {
+                x[u] = load4_f32(tile + kLanes * u);
+                base[u] = pos0 + static_cast<uint32_t>(kLanes * u);
+              }
+              q.template offer_tile<U>(x, base);
+            } else {
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                const uint32_t off = hoff + 4u * tid + static_cast<uint32_t>(kLanes * u);
+                if (off < c)
+                  q.offer4(load4_f32(tile + kLanes * u), pos0 + static_cast<uint32_t>(kLanes * u));
+              }
             }
           }
         } else {
-          select_tile_sparse<KB>(q, ring + static_cast<size_t>(st) * kTile, c,
-                                 static_cast<uint32_t>(a) + done, nq);
+#pragma unroll
+          for (int h = 0; h < kTileElems / kTile; ++h) {
+            const uint32_t hoff = static_cast<uint32_t>(h * kTile);
+            if (hoff < c)
+              select_tile_sparse<KB, T>(q, stage_tile + hoff, c - hoff,
+                                        static_cast<uint32_t>(a) + done + hoff, nq);
+          }
         }
       }
       __syncwarp();
@@ -267,14 +306,14 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs 
         if (v < nq) q.store(v, lanebuf + static_cast<size_t>(tid + kThreads * v) * KB);
     }
     group_sync(kThreads);
-    finish_piece<KB, kGatherInput>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
-                                   p.x + row0, p.out_vals, p.out_idx, piece_flag, nl);
+    finish_piece<KB, kGatherInput, T>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
+                                      p.x + row0, p.out_vals, p.out_idx, piece_flag, nl);
     group_sync(kThreads);
   }
 }
 
-template <int KB>
-__global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, int cand_cap) {
+template <typename T, int KB>
+__global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs<T> p, int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];
   const SelectSmem L{0, KB, cand_cap, kLanes};
   uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem);
@@ -298,7 +337,7 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, 
     const int64_t a = g - row0;
     const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
     const int64_t len = pend - g;
-    const float* src = p.x + g;
+    const T* src = p.x + g;
     q.reset();
     constexpr int U = 4;  // stripes in flight per thread
     for (int64_t base = 0; base < len; base += static_cast<int64_t>(W) * U) {
@@ -309,7 +348,7 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, 
         for (int w = 0; w < 4; ++w) {
           const int l = tid + kThreads * w;
           const int64_t off = base + static_cast<int64_t>(W) * u + l;
-          v[u][w] = (l < W && off < len) ? __ldg(src + off) : __uint_as_float(0xff800000u);
+          v[u][w] = (l < W && off < len) ? to_f32(src[off]) : __uint_as_float(0xff800000u);
         }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -332,8 +371,8 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs p, 
     for (int w = 0; w < 4; ++w)
       q.store(w, lanebuf + static_cast<size_t>(tid + kThreads * w) * KB);
     group_sync(kThreads);
-    finish_piece<KB, kGatherInput>(rs, b, p.k, r, a, len, lanebuf, cand, p.x + row0, p.out_vals,
-                                   p.out_idx, &piece_flag);
+    finish_piece<KB, kGatherInput, T>(rs, b, p.k, r, a, len, lanebuf, cand, p.x + row0, p.out_vals,
+                                      p.out_idx, &piece_flag);
     group_sync(kThreads);
     g = pend;
   }

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kExactThreads) exact_topk_kernel(const float* 
     uint64_t* s = reinterpret_cast<uint64_t*>(smem);
     const int nn = static_cast<int>(n);
     for (int i = tid; i < nn; i += T) s[i] = pack(order_key(__ldg(row + i)), i);
-    finalize_row<kGatherInput>(s, nn, k, row, ov, oi, T);
+    finalize_row<kGatherInput, float>(s, nn, k, row, ov, oi, T);
     return;
   }
 
@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kExactThreads) exact_topk_kernel(const float* 
     // Every element is selected; the sort orders them and pads the rest.
     const int nn = static_cast<int>(n);
     for (int i = tid; i < nn; i += T) sel[i] = pack(order_key(__ldg(row + i)), i);
-    finalize_row<kGatherInput>(sel, nn, k, row, ov, oi, T);
+    finalize_row<kGatherInput, float>(sel, nn, k, row, ov, oi, T);
     return;
   }
 
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kExactThreads) exact_topk_kernel(const float* 
     }
   }
   __syncthreads();
-  finalize_row<kGatherInput>(sel, k, k, row, ov, oi, T);
+  finalize_row<kGatherInput, float>(sel, k, k, row, ov, oi, T);
 }
 
 }  // namespace tk

@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kScorePipeThreads, 2)
 #pragma unroll
     for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
     group_sync(kThreads);
-    finish_piece<KB, kFromKey>(rs, p.b, p.k, r, a, len, lanebuf, cand, nullptr, p.out_vals,
+    finish_piece<KB, kFromKey, float>(rs, p.b, p.k, r, a, len, lanebuf, cand, nullptr, p.out_vals,
                                p.out_idx, piece_flag);
     group_sync(kThreads);
     g = pend;

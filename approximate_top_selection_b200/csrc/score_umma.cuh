@@ -466,7 +466,7 @@ __global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64
     for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
   }
   group_sync(kThreads);
-  stage2<kFromKey>(cand, b * KB, k, nullptr, out_vals + r * k, out_idx + r * k);
+  stage2<kFromKey, float>(cand, b * KB, k, nullptr, out_vals + r * k, out_idx + r * k);
 }
 
 }  // namespace tk

@@ -291,16 +291,31 @@ __device__ __forceinline__ void block_sort_desc(uint64_t (&v)[EPT], uint64_t* xc
 
 // Value of an output candidate: from its key, except that a zero or NaN is
 // re-read from the input row so that -0.0 and NaN payloads keep their bits.
-template <int VS>
-__device__ __forceinline__ float candidate_value(uint64_t p, const float* xrow) {
-  float v = key_value(packed_key(p));
-  if (VS == 0 && (v == 0.0f || v != v)) v = __ldg(xrow + packed_idx(p));
-  return v;
+// V is the element type of the output: float, or uint16_t holding bf16 bits
+// (a bf16 widened to float is exact, so its upper 16 bits give it back).
+template <int VS, typename V>
+__device__ __forceinline__ V candidate_value(uint64_t p, const V* xrow) {
+  const float v = key_value(packed_key(p));
+  if constexpr (sizeof(V) == 4) {
+    if (VS == 0 && (v == 0.0f || v != v)) return __ldg(xrow + packed_idx(p));
+    return v;
+  } else {
+    if (VS == 0 && (v == 0.0f || v != v)) return xrow[packed_idx(p)];
+    return static_cast<V>(__float_as_uint(v) >> 16);
+  }
 }
 
-template <int EPT, int VS>
-__device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, const float* xrow,
-                                                  float* ov, int32_t* oi) {
+template <typename V>
+__device__ __forceinline__ V negative_infinity() {
+  if constexpr (sizeof(V) == 4)
+    return __int_as_float(0xff800000);
+  else
+    return static_cast<V>(0xff80u);
+}
+
+template <int EPT, int VS, typename V>
+__device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                               int32_t* oi) {
   constexpr int N = kThreads * EPT;
   const int t = threadIdx.x;
   uint64_t v[EPT];
@@ -316,16 +331,16 @@ __device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, con
     const int e = t * EPT + j;
     if (e < k) {
       if (v[j]) {
-        ov[e] = candidate_value<VS>(v[j], xrow);
+        ov[e] = candidate_value<VS, V>(v[j], xrow);
         oi[e] = static_cast<int32_t>(packed_idx(v[j]));
       } else {
-        ov[e] = __int_as_float(0xff800000);
+        ov[e] = negative_infinity<V>();
         oi[e] = -1;
       }
     }
   }
   for (int e = N + t; e < k; e += kThreads) {
-    ov[e] = __int_as_float(0xff800000);
+    ov[e] = negative_infinity<V>();
     oi[e] = -1;
   }
   group_sync(kThreads);
@@ -345,18 +360,18 @@ __host__ __device__ __forceinline__ size_t stage2_bytes(int C) {
   return static_cast<size_t>(sort_capacity(C)) * 8 + kStage2Extra;
 }
 
-template <ValueSource VS>
-__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const float* xrow,
-                                                  float* ov, int32_t* oi);
+template <ValueSource VS, typename V>
+__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                                  int32_t* oi);
 
 // Stage 2 when the candidates far outnumber k: find the k-th largest packed
 // key with 8-bit radix histograms (most significant digit first; keys are
 // unique, so at most 8 passes, and the walk stops as soon as the boundary
 // digit holds exactly the elements still needed), gather the selected keys
 // and sort only those.  Same result as sorting all C and keeping k.
-template <int EPT, int VS>
-__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const float* xrow,
-                                                 float* ov, int32_t* oi) {
+template <int EPT, int VS, typename V>
+__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                                 int32_t* oi) {
   const int t = threadIdx.x;
   uint32_t* hist = reinterpret_cast<uint32_t*>(cand + sort_capacity(C));  // 256 bins
   int* misc = reinterpret_cast<int*>(hist + 256);                        // digit, above, count, n
@@ -448,30 +463,30 @@ __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, c
   group_sync(kThreads);
   const int kept = misc[3];
   group_sync(kThreads);
-  finalize_row_fast<static_cast<ValueSource>(VS)>(cand, kept, k, xrow, ov, oi);
+  finalize_row_fast<static_cast<ValueSource>(VS), V>(cand, kept, k, xrow, ov, oi);
 }
 
-template <ValueSource VS>
-__device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const float* xrow,
-                                             float* ov, int32_t* oi, int T);
+template <ValueSource VS, typename V>
+__device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                             int32_t* oi, int T);
+
+template <int EPT, int VS, typename V>
+__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                                 int32_t* oi);
 
 // Stage 2 for the streaming kernels (kThreads threads): up to 8 keys per
 // thread are sorted in registers; larger candidate sets use the shared-memory
 // network.
-template <int EPT, int VS>
-__device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const float* xrow,
-                                                 float* ov, int32_t* oi);
-
-template <ValueSource VS>
-__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const float* xrow,
-                                                  float* ov, int32_t* oi) {
+template <ValueSource VS, typename V>
+__device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                                  int32_t* oi) {
   const int ept = sort_capacity(C) / kThreads;
   switch (ept) {
-    case 1: finalize_row_regs<1, VS>(cand, C, k, xrow, ov, oi); break;
-    case 2: finalize_row_regs<2, VS>(cand, C, k, xrow, ov, oi); break;
-    case 4: finalize_row_regs<4, VS>(cand, C, k, xrow, ov, oi); break;
-    case 8: finalize_row_regs<8, VS>(cand, C, k, xrow, ov, oi); break;
-    default: finalize_row<VS>(cand, C, k, xrow, ov, oi, kThreads); break;
+    case 1: finalize_row_regs<1, VS, V>(cand, C, k, xrow, ov, oi); break;
+    case 2: finalize_row_regs<2, VS, V>(cand, C, k, xrow, ov, oi); break;
+    case 4: finalize_row_regs<4, VS, V>(cand, C, k, xrow, ov, oi); break;
+    case 8: finalize_row_regs<8, VS, V>(cand, C, k, xrow, ov, oi); break;
+    default: finalize_row<VS, V>(cand, C, k, xrow, ov, oi, kThreads); break;
   }
 }
 
@@ -479,9 +494,9 @@ __device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, 
 // and writes the first k (Stage 2: only the k best survive when C > k), padding
 // with -inf / -1.  Values either come from the input row (exact input bits)
 // or from the key (fused scores).  cand must have room for next_pow2(C).
-template <ValueSource VS>
-__device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const float* xrow,
-                                             float* ov, int32_t* oi, int T) {
+template <ValueSource VS, typename V>
+__device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const V* xrow, V* ov,
+                                             int32_t* oi, int T) {
   const int N = next_pow2(C);
   for (int i = C + threadIdx.x; i < N; i += T) cand[i] = 0;
   group_sync(T);
@@ -490,15 +505,10 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
     const uint64_t p = s < N ? cand[s] : 0ull;
     if (p) {
       const uint32_t i = packed_idx(p);
-      float v;
-      if (VS == kGatherInput)
-        v = __ldg(xrow + i);
-      else
-        v = key_value(packed_key(p));
-      ov[s] = v;
+      ov[s] = VS == kGatherInput ? xrow[i] : candidate_value<VS, V>(p, xrow);
       oi[s] = static_cast<int32_t>(i);
     } else {
-      ov[s] = __int_as_float(0xff800000);
+      ov[s] = negative_infinity<V>();
       oi[s] = -1;
     }
   }
@@ -507,17 +517,17 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
 
 // Stage 2 entry of the streaming kernels: select first when that shrinks the
 // sort (at least 1024 candidates and k under half of them), else sort all.
-template <ValueSource VS>
-__device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const float* xrow, float* ov,
+template <ValueSource VS, typename V>
+__device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xrow, V* ov,
                                        int32_t* oi) {
   if (C >= 1024 && 2 * k <= C && C <= 16 * kThreads) {
     switch (sort_capacity(C) / kThreads) {
-      case 4: finalize_row_select<4, VS>(cand, C, k, xrow, ov, oi); return;
-      case 8: finalize_row_select<8, VS>(cand, C, k, xrow, ov, oi); return;
-      default: finalize_row_select<16, VS>(cand, C, k, xrow, ov, oi); return;
+      case 4: finalize_row_select<4, VS, V>(cand, C, k, xrow, ov, oi); return;
+      case 8: finalize_row_select<8, VS, V>(cand, C, k, xrow, ov, oi); return;
+      default: finalize_row_select<16, VS, V>(cand, C, k, xrow, ov, oi); return;
     }
   }
-  finalize_row_fast<VS>(cand, C, k, xrow, ov, oi);
+  finalize_row_fast<VS, V>(cand, C, k, xrow, ov, oi);
 }
 
 // ------------------------------------------------------------------ pieces
@@ -538,18 +548,18 @@ __device__ __forceinline__ int64_t cta_start(const RowSplit& rs, int c) {
 // by the first kThreads threads of the CTA.  A whole-row piece runs Stage 2 at
 // once; a partial piece publishes its per-bucket lists and the last piece of
 // the row to finish runs the merge (and clears what it read).
-template <int KB, ValueSource VS>
+template <int KB, ValueSource VS, typename V>
 __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_t a, int64_t len,
-                             const uint64_t* lanebuf, uint64_t* cand, const float* xrow,
-                             float* out_vals, int32_t* out_idx, int* s_flag, int nl = kLanes) {
+                             const uint64_t* lanebuf, uint64_t* cand, const V* xrow, V* out_vals,
+                             int32_t* out_idx, int* s_flag, int nl = kLanes) {
   constexpr int T = kThreads;
   const int C = b * KB;
-  float* ov = out_vals + r * static_cast<int64_t>(k);
+  V* ov = out_vals + r * static_cast<int64_t>(k);
   int32_t* oi = out_idx + r * static_cast<int64_t>(k);
   if (a == 0 && len == rs.n) {
     merge_lanes<KB>(lanebuf, b, 0, cand, T, nl);
     group_sync(T);
-    stage2<VS>(cand, C, k, xrow, ov, oi);
+    stage2<VS, V>(cand, C, k, xrow, ov, oi);
     return;
   }
   const int64_t row0 = r * rs.n;
@@ -588,7 +598,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
     for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
   }
   group_sync(T);
-  stage2<VS>(cand, C, k, xrow, ov, oi);
+  stage2<VS, V>(cand, C, k, xrow, ov, oi);
   if (threadIdx.x == 0) rs.tickets[r] = 0u;  // leave the workspace zeroed
 }
 

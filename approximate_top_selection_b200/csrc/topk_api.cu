@@ -189,24 +189,24 @@ int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, 
   return static_cast<int>(G);
 }
 
-template <int KB>
+template <typename T, int KB>
 int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
   const int C = b * KB;
   pl->cand_cap = sort_capacity(C);
-  pl->align = fast ? 4 : 1;
+  pl->align = fast ? Elem<T>::kAlign : 1;
   pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap, select_lanes(KB, b)}, 2) : 0;
   int per_sm = 0;
   if (fast) {
     SelectSmem L{pl->stages, KB, pl->cand_cap, select_lanes(KB, b)};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
-    int rc = occupancy(bucket_select_tma<KB>, kPipeThreads, pl->smem, &per_sm);
+    int rc = occupancy(bucket_select_tma<T, KB>, kPipeThreads, pl->smem, &per_sm);
     if (rc) return rc;
   } else {
     SelectSmem L{0, KB, pl->cand_cap, kLanes};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
-    int rc = occupancy(bucket_select_general<KB>, kThreads, pl->smem, &per_sm);
+    int rc = occupancy(bucket_select_general<T, KB>, kThreads, pl->smem, &per_sm);
     if (rc) return rc;
   }
   const int64_t E = rows * n;
@@ -217,13 +217,14 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
   return TOPK_OK;
 }
 
+template <typename T = float>
 int plan_select(bool fast, int64_t rows, int64_t n, int b, int kb, const DeviceInfo& dev,
                 Plan* pl) {
   switch (kb) {
-    case 1: return plan_select_kb<1>(fast, rows, n, b, dev, pl);
-    case 2: return plan_select_kb<2>(fast, rows, n, b, dev, pl);
-    case 3: return plan_select_kb<3>(fast, rows, n, b, dev, pl);
-    case 4: return plan_select_kb<4>(fast, rows, n, b, dev, pl);
+    case 1: return plan_select_kb<T, 1>(fast, rows, n, b, dev, pl);
+    case 2: return plan_select_kb<T, 2>(fast, rows, n, b, dev, pl);
+    case 3: return plan_select_kb<T, 3>(fast, rows, n, b, dev, pl);
+    case 4: return plan_select_kb<T, 4>(fast, rows, n, b, dev, pl);
   }
   return TOPK_EINVAL;
 }
@@ -273,8 +274,11 @@ int check_common(int64_t rows, int64_t n, int k, int b, int kb) {
   return TOPK_OK;
 }
 
-bool select_fast(const float* x, int64_t n, int b) {
-  return aligned16(x) && (n % 4) == 0 && (kLanes % b) == 0;
+// The TMA kernel needs 16-byte aligned rows (bulk copies) and b | 1024 (each
+// register queue sees a single bucket).
+template <typename T>
+bool select_fast(const T* x, int64_t n, int b) {
+  return aligned16(x) && (n % Elem<T>::kAlign) == 0 && (kLanes % b) == 0;
 }
 
 RowSplit make_split(const Plan& pl, int64_t rows, int64_t n, void* ws) {
@@ -332,13 +336,67 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_status();
 }
 
-template <int KB>
-int launch_select_kb(bool fast, const Plan& pl, const SelectArgs& a, cudaStream_t st) {
+template <typename T, int KB>
+int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
   if (fast)
-    return launch_pdl(bucket_select_tma<KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
+    return launch_pdl(bucket_select_tma<T, KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
                       pl.stages, pl.cand_cap);
-  return launch_pdl(bucket_select_general<KB>, dim3(pl.G), dim3(kThreads), pl.smem, st, a,
+  return launch_pdl(bucket_select_general<T, KB>, dim3(pl.G), dim3(kThreads), pl.smem, st, a,
                     pl.cand_cap);
+}
+
+template <typename T>
+int launch_select(int kb, bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
+  switch (kb) {
+    case 1: return launch_select_kb<T, 1>(fast, pl, a, st);
+    case 2: return launch_select_kb<T, 2>(fast, pl, a, st);
+    case 3: return launch_select_kb<T, 3>(fast, pl, a, st);
+    default: return launch_select_kb<T, 4>(fast, pl, a, st);
+  }
+}
+
+// topk_bucketed for either element type.
+template <typename T>
+int run_bucketed(const T* scores, int64_t rows, int64_t n, int k, int b, int kb, T* out_vals,
+                 int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
+  int rc = check_common(rows, n, k, b, kb);
+  if (rc) return rc;
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev))) return rc;
+  const bool fast = select_fast(scores, n, b);
+  Plan pl;
+  if ((rc = plan_select<T>(fast, rows, n, b, kb, dev, &pl))) return rc;
+  if (plan_needs_workspace(pl, rows, n)) {
+    if (!workspace || workspace_bytes < pl.workspace()) return TOPK_EWORKSPACE;
+    if (!aligned16(workspace)) return TOPK_EINVAL;
+  }
+  SelectArgs<T> a;
+  a.x = scores;
+  a.k = k;
+  a.b = b;
+  a.out_vals = out_vals;
+  a.out_idx = out_idx;
+  a.rs = make_split(pl, rows, n, workspace);
+  return launch_select<T>(kb, fast, pl, a, static_cast<cudaStream_t>(stream));
+}
+
+// Workspace of topk_bucketed for either element type: enough for the fast and
+// the general plan, whichever the pointer's alignment selects.
+template <typename T>
+size_t bucketed_workspace(int64_t rows, int64_t n, int b, int kb, const DeviceInfo& dev) {
+  Plan p1, p2;
+  size_t need = 0;
+  bool any = false;
+  if (plan_select<T>(true, rows, n, b, kb, dev, &p1) == TOPK_OK) {
+    need = p1.workspace();
+    any = true;
+  }
+  if (plan_select<T>(false, rows, n, b, kb, dev, &p2) == TOPK_OK) {
+    need = std::max(need, p2.workspace());
+    any = true;
+  }
+  return any ? need : 0;
 }
 
 template <int KB, int D>
@@ -504,15 +562,8 @@ size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int k
   Plan pl;
   if (op == TOPK_OP_EXACT) return 0;
   if (check_common(rows, n, k, b, kb)) return 0;
-  if (op == TOPK_OP_BUCKETED) {
-    // Size for the slower-path plan too so one workspace fits either path.
-    Plan p2;
-    if (plan_select(true, rows, n, b, kb, dev, &pl) && plan_select(false, rows, n, b, kb, dev, &pl))
-      return 0;
-    if (plan_select(false, rows, n, b, kb, dev, &p2) == TOPK_OK)
-      return std::max(pl.workspace(), p2.workspace());
-    return pl.workspace();
-  }
+  if (op == TOPK_OP_BUCKETED) return bucketed_workspace<float>(rows, n, b, kb, dev);
+  if (op == TOPK_OP_BUCKETED_BF16) return bucketed_workspace<uint16_t>(rows, n, b, kb, dev);
   if (op == TOPK_OP_SCORE) {
     if (kLanes % b) return 0;
     if (plan_score(rows, n, b, kb, d, dev, &pl)) return 0;
@@ -526,32 +577,15 @@ size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int k
 int topk_bucketed(const float* scores, int64_t rows, int64_t n, int k, int b, int kb,
                   float* out_vals, int32_t* out_idx, void* workspace, size_t workspace_bytes,
                   void* stream) {
-  if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
-  int rc = check_common(rows, n, k, b, kb);
-  if (rc) return rc;
-  DeviceInfo dev;
-  if ((rc = current_device_info(&dev))) return rc;
-  const bool fast = select_fast(scores, n, b);
-  Plan pl;
-  if ((rc = plan_select(fast, rows, n, b, kb, dev, &pl))) return rc;
-  if (plan_needs_workspace(pl, rows, n)) {
-    if (!workspace || workspace_bytes < pl.workspace()) return TOPK_EWORKSPACE;
-    if (!aligned16(workspace)) return TOPK_EINVAL;
-  }
-  SelectArgs a;
-  a.x = scores;
-  a.k = k;
-  a.b = b;
-  a.out_vals = out_vals;
-  a.out_idx = out_idx;
-  a.rs = make_split(pl, rows, n, workspace);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (kb) {
-    case 1: return launch_select_kb<1>(fast, pl, a, st);
-    case 2: return launch_select_kb<2>(fast, pl, a, st);
-    case 3: return launch_select_kb<3>(fast, pl, a, st);
-    default: return launch_select_kb<4>(fast, pl, a, st);
-  }
+  return run_bucketed<float>(scores, rows, n, k, b, kb, out_vals, out_idx, workspace,
+                             workspace_bytes, stream);
+}
+
+int topk_bucketed_bf16(const uint16_t* scores, int64_t rows, int64_t n, int k, int b, int kb,
+                       uint16_t* out_vals, int32_t* out_idx, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  return run_bucketed<uint16_t>(scores, rows, n, k, b, kb, out_vals, out_idx, workspace,
+                                workspace_bytes, stream);
 }
 
 int topk_bucketed_noalloc(const float* scores, int64_t rows, int64_t n, int k, int b, int kb,
@@ -563,7 +597,7 @@ int topk_bucketed_noalloc(const float* scores, int64_t rows, int64_t n, int k, i
   if ((rc = current_device_info(&dev))) return rc;
   const bool fast = select_fast(scores, n, b);
   Plan pl;
-  if ((rc = plan_select(fast, rows, n, b, kb, dev, &pl))) return rc;
+  if ((rc = plan_select<float>(fast, rows, n, b, kb, dev, &pl))) return rc;
   void* scratch = nullptr;
   if ((rc = noalloc_scratch_ptr(&scratch))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -572,19 +606,14 @@ int topk_bucketed_noalloc(const float* scores, int64_t rows, int64_t n, int k, i
     // The tickets must start at zero whatever an earlier call left behind.
     if (cudaMemsetAsync(scratch, 0, pl.ws_tickets, st) != cudaSuccess) return TOPK_ECUDA;
   }
-  SelectArgs a;
+  SelectArgs<float> a;
   a.x = scores;
   a.k = k;
   a.b = b;
   a.out_vals = out_vals;
   a.out_idx = out_idx;
   a.rs = make_split(pl, rows, n, scratch);
-  switch (kb) {
-    case 1: return launch_select_kb<1>(fast, pl, a, st);
-    case 2: return launch_select_kb<2>(fast, pl, a, st);
-    case 3: return launch_select_kb<3>(fast, pl, a, st);
-    default: return launch_select_kb<4>(fast, pl, a, st);
-  }
+  return launch_select<float>(kb, fast, pl, a, st);
 }
 
 int topk_exact(const float* scores, int64_t rows, int64_t n, int k, float* out_vals,

@@ -54,6 +54,9 @@ for _b in (128, 256, 512):
     for _kb in (1, 2, 4):
         CONFIGS["long-b%d-kb%d" % (_b, _kb)] = dict(kind="select", rows=256, n=131072, k=512,
                                                     b=_b, kb=_kb, dist="uniform")
+# bfloat16 score rows (the page's Fig. 10 repeats its configurations in bf16)
+for _name in ("vocab", "long-b128-kb1", "long-b256-kb2", "long-b512-kb4"):
+    CONFIGS[_name + "-bf16"] = dict(CONFIGS[_name], dtype="bf16")
 
 
 def _peaks():
@@ -155,7 +158,9 @@ class Workload:
                 self.x = inputs.vocab_logits(c["rows"], c["n"], seed, device=device)
             else:
                 self.x = inputs.uniform_rows(c["rows"], c["n"], seed, device=device)
-            self.in_bytes = self.x.numel() * 4
+            if c.get("dtype") == "bf16":
+                self.x = self.x.to(torch.bfloat16)
+            self.in_bytes = self.x.numel() * self.x.element_size()
         self.out_bytes = self.rows * c["k"] * 8
         self.bytes = self.in_bytes + self.out_bytes
         self.larger_than_l2 = self.in_bytes > 126 * 2 ** 20
@@ -327,7 +332,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "bf16" if w.cfg.get("dtype") == "bf16" else "f32",
         "data": "synthetic (seeded; shapes of the pages' workloads)",
         "config": dict(w.describe(), l2="inputs larger than L2" if nrot == 1 else
                        "%d rotating input copies (%.0f MiB) defeat L2" %

@@ -53,7 +53,8 @@ typedef enum {
 typedef enum {
     TOPK_OP_BUCKETED = 0,
     TOPK_OP_EXACT = 1,
-    TOPK_OP_SCORE = 2
+    TOPK_OP_SCORE = 2,
+    TOPK_OP_BUCKETED_BF16 = 3
 } topk_op;
 
 /* Bytes of workspace a call of `op` with these sizes needs on the current
@@ -74,6 +75,21 @@ size_t topk_workspace_bytes(int op, int64_t rows, int64_t n, int k, int b, int k
 int topk_bucketed(const float *scores_dev, int64_t rows, int64_t n, int k, int b, int kb,
                   float *out_vals_dev, int32_t *out_idx_dev, void *workspace_dev,
                   size_t workspace_bytes, void *stream);
+
+/* topk_bucketed on bfloat16 score rows: the same selection on half the bytes
+ * (the page compares the two precisions in Fig. 10, "Bandwidth comparison for
+ * bfloat16 values").
+ *   scores_dev   [rows x n] bf16 (raw 16-bit patterns).
+ *   out_vals_dev [rows x k] bf16: the selected scores, input bits unchanged
+ *                (padding slots hold -inf, 0xFF80).
+ * bf16 values are ordered as the floats they represent, with the same total
+ * order (ties by lowest index, -0 ties +0, NaN above +inf).  Fast path: n % 8
+ * == 0, 16-byte aligned rows, b dividing 1024.  Workspace:
+ * topk_workspace_bytes(TOPK_OP_BUCKETED_BF16, ...); other arguments and
+ * errors as topk_bucketed. */
+int topk_bucketed_bf16(const uint16_t *scores_dev, int64_t rows, int64_t n, int k, int b, int kb,
+                       uint16_t *out_vals_dev, int32_t *out_idx_dev, void *workspace_dev,
+                       size_t workspace_bytes, void *stream);
 
 /* Exact top-k of every row under the total order above: the baseline the
  * page compares against (Fig. 1, "exact top-k implementations") and the

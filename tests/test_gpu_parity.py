@@ -316,3 +316,41 @@ def test_link_config_full(oracle_mod):
     sampled query rows against the fp64 oracle."""
     Q, K = inputs.link_inputs(1024, 1 << 20, 256, inputs.SEEDS["link"], device=DEV)
     check_scores(Q, K, 100, 1024, 1, oracle_mod, rows_subset=[0, 127, 128, 500, 1023])
+
+
+# ------------------------------------------------------------------ bfloat16 rows
+def _bf16_check(x_bf16: torch.Tensor, k, b, kb, oracle_mod, x_dev=None):
+    """bf16 rows: the oracle selects on the exactly widened fp32 values; the
+    GPU must return the same indices and the same bf16 bits."""
+    x_dev = x_bf16.to(DEV) if x_dev is None else x_dev
+    v, i = atk.topk_bucketed(x_dev, k, b, kb)
+    assert v.dtype == torch.bfloat16
+    torch.cuda.synchronize()
+    xf = x_bf16.float().numpy()
+    ov, oi = oracle_mod.bucketed(xf, k, b, kb)
+    assert np.array_equal(i.cpu().numpy(), oi), "bf16 index mismatch (k=%d b=%d kb=%d)" % (k, b, kb)
+    got = v.cpu().view(torch.int16).numpy().view(np.uint16)
+    want = (ov.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(got, want), "bf16 value bits differ"
+
+
+@pytest.mark.parametrize("kb", [1, 2, 3, 4])
+def test_bf16_rows(oracle_mod, kb):
+    """bf16 has 8 mantissa bits: rows are full of ties, the lowest index wins."""
+    x = inputs.normal_rows(6, 65536, 300 + kb).to(torch.bfloat16)
+    for (k, b) in [(64, 128), (512, 256), (50, 512), (100, 1024)]:
+        _bf16_check(x, k, b, kb, oracle_mod)
+
+
+def test_bf16_special_values_and_general_path(oracle_mod):
+    x = inputs.special_rows(8, 8192, 71).to(torch.bfloat16)
+    _bf16_check(x, 100, 64, 2, oracle_mod)
+    x = inputs.normal_rows(3, 3001, 72).to(torch.bfloat16)  # n % 8 != 0: general path
+    _bf16_check(x, 60, 100, 3, oracle_mod)
+    x = inputs.normal_rows(2, 500000, 73).to(torch.bfloat16)  # split rows
+    _bf16_check(x, 300, 512, 2, oracle_mod)
+
+
+def test_bf16_vocab_config(oracle_mod):
+    x = inputs.vocab_logits(256, 131072, inputs.SEEDS["vocab"]).to(torch.bfloat16)
+    _bf16_check(x, 50, 512, 1, oracle_mod)
