@@ -87,15 +87,13 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
   constexpr int U = kTile / kThreads;  // 32 elements per thread (8192 per call)
   const int t = threadIdx.x;
   float x[U];
-  float m = __int_as_float(0x7f800000);
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const bool valid = static_cast<uint32_t>(t + kThreads * u) < c;
     x[u] = valid ? to_f32(tile[t + kThreads * u]) : __int_as_float(0x7f800000);
-    m = fmin_nan(m, x[u]);
   }
   const uint32_t base = pos_tile + static_cast<uint32_t>(t);
-  if (!(m > __int_as_float(0xff800000))) {
+  if (!(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
     // NaN or -inf somewhere in this thread's elements: exact update, in order.
 #pragma unroll
     for (int u = 0; u < U; ++u) {

@@ -61,6 +61,30 @@ __device__ __forceinline__ void pdl_wait_then_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Three-input form (sm_100).
+__device__ __forceinline__ float fmin3_nan(float a, float b, float c) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// NaN-keeping minimum of N values (three-input steps).
+template <int N>
+__device__ __forceinline__ float min_nan_all(const float (&v)[N]) {
+  float m[(N + 2) / 3];
+#pragma unroll
+  for (int i = 0; i < (N + 2) / 3; ++i) {
+    const float a = v[3 * i];
+    const float b = 3 * i + 1 < N ? v[3 * i + 1] : a;
+    const float c = 3 * i + 2 < N ? v[3 * i + 2] : a;
+    m[i] = fmin3_nan(a, b, c);
+  }
+  if constexpr ((N + 2) / 3 == 1)
+    return m[0];
+  else
+    return min_nan_all<(N + 2) / 3>(m);
+}
+
 // ---------------------------------------------------------------- mbarrier / bulk copy
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -198,10 +198,10 @@ template <int KB, int NQ, int QI>
 __device__ __forceinline__ void umma_feed_bucket(BucketQueues<NQ, KB>& q, const uint32_t (&r)[32],
                                                  int t0, int T, uint32_t b, uint32_t jb, int64_t row,
                                                  int64_t rows, int64_t n, float* out_scores) {
-  float m = __uint_as_float(r[0]);
+  float all[32];
 #pragma unroll
-  for (int i = 1; i < 32; ++i) m = fmin_nan(m, __uint_as_float(r[i]));
-  const bool special = !(m > __int_as_float(0xff800000));
+  for (int i = 0; i < 32; ++i) all[i] = __uint_as_float(r[i]);
+  const bool special = !(min_nan_all<32>(all) > __int_as_float(0xff800000));
   const int valid = T - t0 < 32 ? T - t0 : 32;  // stripes of this tile inside the tensor
   if (out_scores != nullptr && row < rows) {
 #pragma unroll
@@ -246,7 +246,6 @@ __global__ void __launch_bounds__(umma_threads(KB), 1)
                       UmmaArgs p) {
   constexpr int kEpiWarps = umma_epi_warps(KB);
   constexpr int H = kEpiWarps / 4;             // warps sharing one TMEM lane quarter
-  constexpr int kColsPerWarp = kUmmaN / H;     // accumulator columns each of them drains
   using L = UmmaSmem<D>;
   constexpr int kChunks = L::kChunks;
   constexpr uint32_t kIdesc = umma_idesc_bf16(kUmmaM, kUmmaN);

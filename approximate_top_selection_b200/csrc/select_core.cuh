@@ -127,15 +127,15 @@ struct Queues {
   // min over all 4U values decides whether any of them is NaN or -inf.
   template <int U>
   __device__ __forceinline__ void offer_tile(const float4 (&x)[U], const uint32_t (&base)[U]) {
-    float m[U];
+    float all[4 * U];
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      m[u] = fmin_nan(fmin_nan(x[u].x, x[u].y), fmin_nan(x[u].z, x[u].w));
-#pragma unroll
-    for (int w = 1; w < U; w <<= 1)
-#pragma unroll
-      for (int u = 0; u + w < U; u += 2 * w) m[u] = fmin_nan(m[u], m[u + w]);
-    const bool sp = !(m[0] > __int_as_float(0xff800000));
+    for (int u = 0; u < U; ++u) {
+      all[4 * u] = x[u].x;
+      all[4 * u + 1] = x[u].y;
+      all[4 * u + 2] = x[u].z;
+      all[4 * u + 3] = x[u].w;
+    }
+    const bool sp = !(min_nan_all<4 * U>(all) > __int_as_float(0xff800000));
     if (!sp) {
 #pragma unroll
       for (int u = 0; u < U; ++u) fast4(x[u], base[u]);
