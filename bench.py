@@ -199,6 +199,44 @@ def _rotations(w: Workload) -> int:
     return 1 if w.larger_than_l2 else max(2, math.ceil(3 * 126 * 2 ** 20 / w.in_bytes))
 
 
+def _time_ms(fn, steps: int, warmup: int = 3) -> float:
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def exact_context(w: Workload, ms_bucketed: float, steps: int = 20):
+    """Context for the page's claim (bucketed vs exact top-k): on the same
+    resident input, this library's exact top-k and torch.topk (for the fused
+    workloads: the PyTorch scores, materialised, then torch.topk)."""
+    import approximate_top_selection_b200 as atk
+
+    c = w.cfg
+    out = {"bucketed_ms": ms_bucketed}
+    if c["kind"] == "select":
+        x = w.x.float() if w.x.dtype != torch.float32 else w.x
+        out["exact_topk_ms"] = _time_ms(lambda: atk.topk_exact(x, c["k"]), steps)
+        out["torch_topk_ms"] = _time_ms(lambda: torch.topk(w.x, c["k"], dim=1), steps)
+    else:
+        if w.K.dim() == 3:
+            fn = lambda: torch.topk(torch.bmm(w.K, w.q[:, :, None]).squeeze(-1).float(),  # noqa: E731
+                                    c["k"], dim=1)
+        else:
+            fn = lambda: torch.topk((w.q @ w.K.T).float(), c["k"], dim=1)  # noqa: E731
+        out["torch_scores_then_topk_ms"] = _time_ms(fn, max(3, steps // 4))
+    for key in list(out):
+        if key != "bucketed_ms":
+            out["speedup_vs_" + key[:-3]] = out[key] / ms_bucketed
+    return out
+
+
 def recall_report(w: Workload):
     """Recall of the step's selection against exact top-k on the same scores."""
     import approximate_top_selection_b200 as atk
@@ -213,7 +251,8 @@ def recall_report(w: Workload):
         rows = min(w.rows, 256)
         s = w.x[:rows]
         _, bi = atk.topk_bucketed(s, c["k"], c["b"], c["kb"])
-    _, ei = atk.topk_exact(s, c["k"])
+    # bf16 widens to fp32 exactly, so the exact selection sees the same values
+    _, ei = atk.topk_exact(s.float() if s.dtype != torch.float32 else s, c["k"])
     r = rc.recall(bi.cpu().numpy(), ei.cpu().numpy())
     n = c["n"]
     out = {"mean": float(r.mean()), "rows": rows, "eq1": rc.eq1_expected_recall(c["k"], c["b"], c["kb"])}
@@ -344,6 +383,8 @@ def run_ours(args, world, rank, local):
     }
     if not args.no_recall:
         line["recall"] = recall_report(w)
+    if args.context:
+        line["context"] = exact_context(w, ms_step)
     if not args.no_e2e:
         line["e2e"] = e2e(w, args, world)
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -506,6 +547,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-recall", action="store_true")
+    ap.add_argument("--context", action="store_true",
+                    help="also time exact top-k (this library and torch.topk) on the same input")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
