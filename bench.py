@@ -392,27 +392,35 @@ def run_ours(args, world, rank, local):
     return line
 
 
-def _source_hash() -> str:
-    import glob
+# Device sources of each timed kernel: a traffic figure stays valid while these
+# files are unchanged since the capture.
+_KERNEL_SOURCES = {
+    "bucket_select_tma": ("common.cuh", "select_core.cuh", "bucket_select.cuh"),
+    "score_select_gemv": ("common.cuh", "select_core.cuh", "score_gemv.cuh"),
+    "score_select_umma": ("common.cuh", "select_core.cuh", "score_umma.cuh"),
+}
+
+
+def _source_hash(kernel: str) -> str:
     import hashlib
 
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "approximate_top_selection_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for f in _KERNEL_SOURCES.get(kernel, ()):
+        with open(os.path.join(ROOT, "approximate_top_selection_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def _traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernels
-    have not changed since it was taken (else None)."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    device sources have not changed since it was taken (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.md")
     if not os.path.exists(path):
         return None
-    cur = _source_hash()
     for line in open(path):
         cells = [c.strip() for c in line.strip().strip("|").split("|")]
-        if len(cells) >= 4 and cells[0] == workload and cells[2] == cur:
+        if len(cells) >= 4 and cells[0] == workload and cells[1] in _KERNEL_SOURCES \
+                and cells[2] == _source_hash(cells[1]):
             try:
                 return int(cells[3])
             except ValueError:
