@@ -58,6 +58,9 @@ def load_library():
             lib.topk_bucketed_bf16.restype = i32
             lib.topk_bucketed_noalloc.argtypes = [p, i64, i64, i32, i32, i32, p, p, p]
             lib.topk_bucketed_noalloc.restype = i32
+            lib.topk_bucketed_merge.argtypes = [p, p, i32, i64, i32, ctypes.POINTER(ctypes.c_int64),
+                                                i64, i32, i32, i32, p, p, p]
+            lib.topk_bucketed_merge.restype = i32
             lib.topk_status_string.argtypes = [i32]
             lib.topk_status_string.restype = ctypes.c_char_p
             lib.topk_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -213,6 +216,38 @@ def topk_exact(scores: torch.Tensor, k: int, *, out_vals=None, out_idx=None, str
         st = lib.topk_exact(scores.data_ptr(), rows, n, k, out_vals.data_ptr(),
                             out_idx.data_ptr(), None, 0, sh)
     _check(st, "topk_exact")
+    return out_vals, out_idx
+
+
+def topk_bucketed_merge(vals: torch.Tensor, idx: torch.Tensor, n_total: int, k: int, b: int,
+                        kb: int, *, part_offsets=None, out_vals=None, out_idx=None, stream=None):
+    """Bucketed top-k over candidate lists (bucket = global index mod b).
+
+    vals: [parts, rows, m] float32, idx: [parts, rows, m] int32 (-1 = empty),
+    both on the GPU; part_offsets: `parts` integers added to each part's
+    indices (default 0).  With each part's lists = topk_bucketed of a column
+    slice of the same rows, the result is topk_bucketed of the whole rows.
+    """
+    lib = load_library()
+    _cuda(vals, "vals", torch.float32)
+    _cuda(idx, "idx", torch.int32)
+    if vals.dim() == 2:
+        vals, idx = vals[None], idx[None]
+    if vals.dim() != 3 or tuple(idx.shape) != tuple(vals.shape):
+        raise ValueError("vals and idx must both be [parts, rows, m]")
+    if idx.device != vals.device:
+        raise ValueError("vals and idx must be on the same device")
+    parts, rows, m = vals.shape
+    offs = [0] * parts if part_offsets is None else [int(o) for o in part_offsets]
+    if len(offs) != parts:
+        raise ValueError("part_offsets needs one entry per part")
+    c_offs = (ctypes.c_int64 * parts)(*offs)
+    with torch.cuda.device(vals.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, vals.device, out_vals, out_idx)
+        st = lib.topk_bucketed_merge(vals.data_ptr(), idx.data_ptr(), parts, rows, m, c_offs,
+                                     n_total, k, b, kb, out_vals.data_ptr(), out_idx.data_ptr(), sh)
+    _check(st, "topk_bucketed_merge")
     return out_vals, out_idx
 
 

@@ -12,6 +12,7 @@
 #include "../../include/topk_b200.h"
 #include "bucket_select.cuh"
 #include "exact_topk.cuh"
+#include "merge_select.cuh"
 #include "score_gemv.cuh"
 #include "score_umma.cuh"
 
@@ -633,6 +634,53 @@ int topk_exact(const float* scores, int64_t rows, int64_t n, int k, float* out_v
   if ((rc = prepare_kernel(exact_topk_kernel))) return rc;
   return launch_pdl(exact_topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(kExactThreads), smem,
                     static_cast<cudaStream_t>(stream), scores, n, k, L.sel_cap, out_vals, out_idx);
+}
+
+int topk_bucketed_merge(const float* vals, const int32_t* idx, int parts, int64_t rows, int m,
+                        const int64_t* part_offset, int64_t n_total, int k, int b, int kb,
+                        float* out_vals, int32_t* out_idx, void* stream) {
+  if (!vals || !idx || !out_vals || !out_idx) return TOPK_EINVAL;
+  if (parts < 1 || m < 1) return TOPK_EINVAL;
+  int rc = check_common(rows, n_total, k, b, kb);
+  if (rc) return rc;
+  if (parts > kMergeMaxParts || rows > 2147483647LL) return TOPK_EUNSUPPORTED;
+  if (static_cast<int64_t>(parts) * m > kMaxElems / rows) return TOPK_EUNSUPPORTED;
+  MergeArgs a{};
+  a.vals = vals;
+  a.idx = idx;
+  a.parts = parts;
+  a.m = m;
+  a.k = k;
+  a.b = b;
+  a.rows = rows;
+  a.n_total = n_total;
+  a.out_vals = out_vals;
+  a.out_idx = out_idx;
+  for (int i = 0; i < parts; ++i) {
+    const int64_t o = part_offset ? part_offset[i] : 0;
+    if (o < 0 || o >= n_total) return TOPK_EINVAL;
+    a.offs[i] = o;
+  }
+  DeviceInfo dev;
+  if ((rc = current_device_info(&dev))) return rc;
+  const size_t smem = stage2_bytes(b * kb);
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(rows)), block(kThreads);
+  switch (kb) {
+    case 1:
+      if ((rc = prepare_kernel(bucket_merge_kernel<1>))) return rc;
+      return launch_pdl(bucket_merge_kernel<1>, grid, block, smem, st, a);
+    case 2:
+      if ((rc = prepare_kernel(bucket_merge_kernel<2>))) return rc;
+      return launch_pdl(bucket_merge_kernel<2>, grid, block, smem, st, a);
+    case 3:
+      if ((rc = prepare_kernel(bucket_merge_kernel<3>))) return rc;
+      return launch_pdl(bucket_merge_kernel<3>, grid, block, smem, st, a);
+    default:
+      if ((rc = prepare_kernel(bucket_merge_kernel<4>))) return rc;
+      return launch_pdl(bucket_merge_kernel<4>, grid, block, smem, st, a);
+  }
 }
 
 int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,

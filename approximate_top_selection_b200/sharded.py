@@ -1,0 +1,74 @@
+"""Rows cut into column slices across ranks (vocabulary- or entity-parallel).
+
+Each rank holds columns [offset, offset + n_local) of the same rows.  It runs
+the bucketed selection on its slice, the (value, index) candidate lists of all
+ranks are all-gathered -- the one exchange of the method when a row is split
+-- and `topk_bucketed_merge` finishes with buckets taken by global index
+modulo b ("Approximate Top-k for Increased Parallelism", pith.science review
+page, "What carries the argument"; "The reading").  The result equals the
+single-pass selection of the whole rows, bit for bit, for any cut points.
+
+A slice's own selection may use local indices: its positions fall into the
+same residue classes as their global indices shifted by one offset, so it
+keeps the same elements; the merge adds the offsets.
+
+The collectives are plain torch.distributed calls (NCCL between GPUs, gloo on
+the host); every rank calls them in the same order.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import _binding
+
+
+def column_slices(n_total: int, world: int) -> list[tuple[int, int]]:
+    """Contiguous (offset, length) slices of [0, n_total), as even as possible."""
+    if world < 1 or n_total < world:
+        raise ValueError("need 1 <= world <= n_total")
+    base, extra = divmod(n_total, world)
+    out, off = [], 0
+    for r in range(world):
+        ln = base + (1 if r < extra else 0)
+        out.append((off, ln))
+        off += ln
+    return out
+
+
+def gather_offsets(offset: int, group=None, device=None) -> list[int]:
+    """Every rank's column offset, in rank order."""
+    world = dist.get_world_size(group)
+    t = torch.tensor([int(offset)], dtype=torch.int64, device=device)
+    parts = [torch.empty_like(t) for _ in range(world)]
+    dist.all_gather(parts, t, group=group)
+    return [int(p.item()) for p in parts]
+
+
+def gather_candidates(vals: torch.Tensor, idx: torch.Tensor, group=None):
+    """All-gather per-rank candidate lists [rows, m] into [world, rows, m]."""
+    world = dist.get_world_size(group)
+    vals, idx = vals.contiguous(), idx.contiguous()
+    out_v = torch.empty((world,) + tuple(vals.shape), dtype=vals.dtype, device=vals.device)
+    out_i = torch.empty((world,) + tuple(idx.shape), dtype=idx.dtype, device=idx.device)
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(out_v, vals, group=group)
+        dist.all_gather_into_tensor(out_i, idx, group=group)
+    else:
+        dist.all_gather(list(out_v.unbind(0)), vals, group=group)
+        dist.all_gather(list(out_i.unbind(0)), idx, group=group)
+    return out_v, out_i
+
+
+def split_row_topk(x_local: torch.Tensor, offset: int, n_total: int, k: int, b: int, kb: int,
+                   group=None):
+    """Bucketed top-k of rows whose columns are spread over the ranks.
+
+    x_local: this rank's [rows, n_local] float32 slice on its GPU, starting at
+    global column `offset`.  Returns (values, global indices) [rows, k] on every
+    rank.
+    """
+    v, i = _binding.topk_bucketed(x_local, k, b, kb)
+    offsets = gather_offsets(offset, group, device=x_local.device)
+    V, I = gather_candidates(v, i, group)
+    return _binding.topk_bucketed_merge(V, I, n_total, k, b, kb, part_offsets=offsets)

@@ -98,6 +98,33 @@ int topk_bucketed_bf16(const uint16_t *scores_dev, int64_t rows, int64_t n, int 
 int topk_exact(const float *scores_dev, int64_t rows, int64_t n, int k, float *out_vals_dev,
                int32_t *out_idx_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
 
+/* Bucketed top-k over candidate lists: the merge step of a row cut into
+ * column slices (several CTAs, or several GPUs that each hold part of a
+ * vocabulary or an entity table).  The bucket of a pair is its GLOBAL index
+ * modulo b, as for a single pass over the whole row ("What carries the
+ * argument"; bucket = i mod b per "The reading"); each bucket keeps its top
+ * kb pairs and the final exact top-k keeps the k best, with the total order
+ * above.  When part p's lists are topk_bucketed of columns
+ * [part_offset[p], part_offset[p] + n_p) of the same rows (local indices),
+ * the result equals topk_bucketed of the whole rows bit for bit.
+ *   vals_dev [parts x rows x m] float32 and idx_dev [parts x rows x m] int32:
+ *                per part and row, m (value, index) pairs; index -1 marks an
+ *                empty slot (as topk_bucketed pads).  Indices of one row must
+ *                be distinct after the offsets are added.
+ *   parts        1 <= parts <= 64 (else TOPK_EUNSUPPORTED).
+ *   part_offset  HOST array [parts] added to every index of that part; NULL
+ *                means all zero.  0 <= part_offset[p] < n_total.
+ *   n_total      length of the whole rows, 1 <= n_total < 2^31.  A pair whose
+ *                global index is >= n_total is skipped and sets
+ *                TOPK_DEV_BAD_INDEX in the device status.
+ *   k, b, kb     as in topk_bucketed; out_vals_dev / out_idx_dev [rows x k]
+ *                best-first with global indices and the input value bits,
+ *                padded with -inf / -1.
+ * No workspace.  Asynchronous on `stream`. */
+int topk_bucketed_merge(const float *vals_dev, const int32_t *idx_dev, int parts, int64_t rows,
+                        int m, const int64_t *part_offset, int64_t n_total, int k, int b, int kb,
+                        float *out_vals_dev, int32_t *out_idx_dev, void *stream);
+
 /* Fused selector: score[r][i] = sum_t q[r][t] * K_r[i][t] (bf16 inputs, fp32
  * accumulation; no 1/sqrt(d) scaling), then topk_bucketed on each row of
  * scores -- the sparse-attention selector that scores the current query
@@ -158,6 +185,7 @@ const char *topk_status_string(int status);
 int topk_device_status(int *status_out);
 
 #define TOPK_DEV_WAIT_TIMEOUT 1 /* a bulk-copy wait in a streaming kernel expired */
+#define TOPK_DEV_BAD_INDEX 2    /* topk_bucketed_merge skipped a pair with index >= n_total */
 
 #ifdef __cplusplus
 }

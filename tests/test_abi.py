@@ -72,6 +72,32 @@ def test_rejects_bad_arguments_on_host(lib):
     assert lib.score_topk(q, 1, 128, p, 8, 0, 1, 1, 1, p, p, None, None, 0, None) == E
 
 
+def test_merge_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    E, U = atk.TOPK_EINVAL, atk.TOPK_EUNSUPPORTED
+    offs = (ctypes.c_int64 * 2)(0, 100)
+    ok = dict(parts=2, rows=1, m=8, n=200, k=4, b=8, kb=1)
+
+    def call(vals=p, idx=p, offsets=offs, out=p, **kw):
+        a = dict(ok, **kw)
+        return lib.topk_bucketed_merge(vals, idx, a["parts"], a["rows"], a["m"], offsets, a["n"],
+                                       a["k"], a["b"], a["kb"], out, p, None)
+
+    assert call(vals=None) == E
+    assert call(idx=None) == E
+    assert call(out=None) == E
+    assert call(parts=0) == E
+    assert call(m=0) == E
+    assert call(rows=0) == E
+    assert call(kb=5) == E
+    assert call(n=0) == E
+    assert call(offsets=(ctypes.c_int64 * 2)(0, 200)) == E   # offset beyond the row
+    assert call(offsets=(ctypes.c_int64 * 2)(-1, 0)) == E
+    assert call(parts=65, offsets=None) == U
+    assert call(b=2048) == U
+    assert call(k=20000) == U
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
 
@@ -79,3 +105,5 @@ def test_binding_refuses_cpu_tensors(lib):
         atk.topk_bucketed(torch.zeros(2, 8), 1, 1, 1)
     with pytest.raises(TypeError):
         atk.topk_exact(torch.zeros(2, 8), 1)
+    with pytest.raises(TypeError):
+        atk.topk_bucketed_merge(torch.zeros(2, 1, 8), torch.zeros(2, 1, 8, dtype=torch.int32), 16, 4, 8, 1)
