@@ -125,17 +125,23 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
       mask[u & 3] |=
           (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[u & 3]) ? (1u << u) : 0u;
   }
+  // Survivors of each queue in turn, re-read from shared memory.
+  const T* tt = tile + t;
 #define TK_SURVIVORS(Q)                                                                   \
   while (mask[Q]) {                                                                       \
     const int u = __ffs(mask[Q]) - 1;                                                     \
     mask[Q] &= mask[Q] - 1u;                                                              \
-    q.template insert_fast<Q>(to_f32(tile[t + kThreads * u]),                             \
+    q.template insert_fast<Q>(to_f32(tt[kThreads * u]),                                   \
                               base + static_cast<uint32_t>(kThreads * u) - (Q));          \
   }
   TK_SURVIVORS(0)
-  TK_SURVIVORS(1)
-  TK_SURVIVORS(2)
-  TK_SURVIVORS(3)
+  if (nq > 1) {
+    TK_SURVIVORS(1)
+  }
+  if (nq > 2) {
+    TK_SURVIVORS(2)
+    TK_SURVIVORS(3)
+  }
 #undef TK_SURVIVORS
 }
 

@@ -376,14 +376,44 @@ __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, c
   uint32_t* hist = reinterpret_cast<uint32_t*>(cand + sort_capacity(C));  // 256 bins
   int* misc = reinterpret_cast<int*>(hist + 256);                        // digit, above, count, n
   uint64_t v[EPT];
+  uint64_t any_bits = 0ull, all_bits = ~0ull;
 #pragma unroll
   for (int j = 0; j < EPT; ++j) {
-    const int e = t * EPT + j;
+    const int e = j * kThreads + t;
     v[j] = e < C ? cand[e] : 0ull;
+    if (v[j] != 0ull) {
+      any_bits |= v[j];
+      all_bits &= v[j];
+    }
   }
-  uint64_t prefix = 0;
+  // The bytes above the highest bit in which the real keys differ are common
+  // to all of them: the digit walk starts below them.
+  uint32_t* red = reinterpret_cast<uint32_t*>(misc + 4);  // OR lo/hi, AND lo/hi
+  if (t == 0) {
+    red[0] = 0u;
+    red[1] = 0u;
+    red[2] = ~0u;
+    red[3] = ~0u;
+  }
+  group_sync(kThreads);
+  {
+    const uint32_t o0 = __reduce_or_sync(0xffffffffu, static_cast<uint32_t>(any_bits));
+    const uint32_t o1 = __reduce_or_sync(0xffffffffu, static_cast<uint32_t>(any_bits >> 32));
+    const uint32_t a0 = __reduce_and_sync(0xffffffffu, static_cast<uint32_t>(all_bits));
+    const uint32_t a1 = __reduce_and_sync(0xffffffffu, static_cast<uint32_t>(all_bits >> 32));
+    if ((t & 31) == 0) {
+      atomicOr(red, o0);
+      atomicOr(red + 1, o1);
+      atomicAnd(red + 2, a0);
+      atomicAnd(red + 3, a1);
+    }
+  }
+  group_sync(kThreads);
+  const uint64_t common_and = red[2] | (static_cast<uint64_t>(red[3]) << 32);
+  const uint64_t differ = (red[0] | (static_cast<uint64_t>(red[1]) << 32)) ^ common_and;
+  int shift = differ ? ((63 - __clzll(static_cast<long long>(differ))) & ~7) : 0;
+  uint64_t prefix = shift < 56 ? (common_and & ~((1ull << (shift + 8)) - 1ull)) : 0ull;
   int need = k;
-  int shift = 56;
   bool all_real = false;
   for (; shift >= 0; shift -= 8) {
     for (int i = t; i < 256; i += kThreads) hist[i] = 0u;
@@ -451,6 +481,7 @@ __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, c
   if (t == 0) misc[3] = 0;
   group_sync(kThreads);
   const int sh = shift < 0 ? 0 : shift;
+  const int lane = t & 31;
 #pragma unroll
   for (int j = 0; j < EPT; ++j) {
     bool sel;
@@ -458,7 +489,15 @@ __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, c
       sel = v[j] != 0ull && (sh == 56 ? true : (v[j] >> (sh + 8)) >= (prefix >> (sh + 8)));
     else
       sel = v[j] != 0ull && (v[j] >> sh) >= (prefix >> sh);
-    if (sel) cand[atomicAdd(misc + 3, 1)] = v[j];
+    // One counter update per warp, not per selected key.
+    const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
+    if (sel_mask) {
+      const int leader = __ffs(sel_mask) - 1;
+      int at = 0;
+      if (lane == leader) at = atomicAdd(misc + 3, __popc(sel_mask));
+      at = __shfl_sync(0xffffffffu, at, leader);
+      if (sel) cand[at + __popc(sel_mask & ((1u << lane) - 1u))] = v[j];
+    }
   }
   group_sync(kThreads);
   const int kept = misc[3];
