@@ -55,6 +55,26 @@ def special_rows(rows: int, n: int, seed: int, with_nan: bool = True) -> torch.T
     return x
 
 
+def ar1_rows(rows: int, n: int, rho: float, seed: int, device="cpu") -> torch.Tensor:
+    """rows x n float32, a stationary AR(1) Gaussian process along each row:
+    x_0 ~ N(0, 1), x_i = rho x_{i-1} + sqrt(1 - rho^2) e_i with e_i iid N(0, 1),
+    so every x_i is N(0, 1) and corr(x_i, x_{i+l}) = rho^l.  The correlated
+    inputs of the page's assignment study (Appendix A.1, Fig. 6: AR(1)
+    multivariate-normal rows); |rho| < 1.
+    """
+    import numpy as np
+    from scipy.signal import lfilter
+
+    if not -1.0 < rho < 1.0:
+        raise ValueError("need |rho| < 1")
+    g = _gen(seed, "cpu")
+    e = torch.randn(rows, n, generator=g, dtype=torch.float64).numpy()
+    start = torch.randn(rows, 1, generator=g, dtype=torch.float64).numpy()  # x_{-1}
+    c = float(np.sqrt(1.0 - rho * rho))
+    x = lfilter([c], [1.0, -rho], e, axis=1, zi=rho * start)[0]
+    return torch.from_numpy(x.astype(np.float32)).to(device)
+
+
 def zipf_permutation(n: int, seed: int, device="cpu") -> torch.Tensor:
     """A seeded permutation rho of [0, n) (token id -> popularity rank)."""
     return torch.randperm(n, generator=_gen(seed ^ 0x5A5A, device), device=device)
