@@ -61,6 +61,11 @@ def load_library():
             lib.topk_bucketed_merge.argtypes = [p, p, i32, i64, i32, ctypes.POINTER(ctypes.c_int64),
                                                 i64, i32, i32, i32, p, p, p]
             lib.topk_bucketed_merge.restype = i32
+            f32 = ctypes.c_float
+            lib.topk_sample_rows.argtypes = [p, p, i64, i32, f32, p, p, p]
+            lib.topk_sample_rows.restype = i32
+            lib.topk_sample.argtypes = [p, i64, i64, i32, i32, i32, f32, p, p, p, p, p, sz, p]
+            lib.topk_sample.restype = i32
             lib.topk_status_string.argtypes = [i32]
             lib.topk_status_string.restype = ctypes.c_char_p
             lib.topk_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -249,6 +254,54 @@ def topk_bucketed_merge(vals: torch.Tensor, idx: torch.Tensor, n_total: int, k: 
                                      n_total, k, b, kb, out_vals.data_ptr(), out_idx.data_ptr(), sh)
     _check(st, "topk_bucketed_merge")
     return out_vals, out_idx
+
+
+def topk_sample_rows(vals: torch.Tensor, idx: torch.Tensor, temperature: float, u: torch.Tensor, *,
+                     out_token=None, stream=None):
+    """One token per row drawn from the softmax (temperature T) of the row's
+    selected logits, by inverse CDF with the given uniforms u [rows]."""
+    lib = load_library()
+    _cuda(vals, "vals", torch.float32)
+    _cuda(idx, "idx", torch.int32)
+    _cuda(u, "u", torch.float32)
+    if vals.dim() != 2 or tuple(idx.shape) != tuple(vals.shape) or u.numel() != vals.shape[0]:
+        raise ValueError("vals, idx must be [rows, k] and u [rows]")
+    rows, k = vals.shape
+    with torch.cuda.device(vals.device):
+        sh = _stream_handle(stream)
+        if out_token is None:
+            out_token = torch.empty(rows, dtype=torch.int32, device=vals.device)
+        _cuda(out_token, "out_token", torch.int32)
+        st = lib.topk_sample_rows(vals.data_ptr(), idx.data_ptr(), rows, k, float(temperature),
+                                  u.data_ptr(), out_token.data_ptr(), sh)
+    _check(st, "topk_sample_rows")
+    return out_token
+
+
+def topk_sample(logits: torch.Tensor, k: int, b: int, kb: int, temperature: float, u: torch.Tensor, *,
+                out_vals=None, out_idx=None, out_token=None, stream=None):
+    """Bucketed top-k of float32 logits [rows, n], then one sampled token per
+    row.  Returns (tokens [rows], values [rows, k], indices [rows, k])."""
+    lib = load_library()
+    _cuda(logits, "logits", torch.float32)
+    _cuda(u, "u", torch.float32)
+    if logits.dim() != 2 or u.numel() != logits.shape[0]:
+        raise ValueError("logits must be [rows, n] and u [rows]")
+    rows, n = logits.shape
+    with torch.cuda.device(logits.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, logits.device, out_vals, out_idx)
+        if out_token is None:
+            out_token = torch.empty(rows, dtype=torch.int32, device=logits.device)
+        _cuda(out_token, "out_token", torch.int32)
+        nbytes = topk_workspace_bytes(TOPK_OP_BUCKETED, rows, n, k, b, kb)
+        ws = _workspace(nbytes, logits.device, sh)
+        st = lib.topk_sample(logits.data_ptr(), rows, n, k, b, kb, float(temperature), u.data_ptr(),
+                             out_token.data_ptr(), out_vals.data_ptr(), out_idx.data_ptr(),
+                             ws.data_ptr() if ws is not None else None,
+                             ws.numel() if ws is not None else 0, sh)
+    _check(st, "topk_sample")
+    return out_token, out_vals, out_idx
 
 
 def score_topk(q: torch.Tensor, K: torch.Tensor, k: int, b: int, kb: int, *,

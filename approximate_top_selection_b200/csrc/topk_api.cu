@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -13,6 +14,7 @@
 #include "bucket_select.cuh"
 #include "exact_topk.cuh"
 #include "merge_select.cuh"
+#include "sample.cuh"
 #include "score_gemv.cuh"
 #include "score_umma.cuh"
 
@@ -681,6 +683,34 @@ int topk_bucketed_merge(const float* vals, const int32_t* idx, int parts, int64_
       if ((rc = prepare_kernel(bucket_merge_kernel<4>))) return rc;
       return launch_pdl(bucket_merge_kernel<4>, grid, block, smem, st, a);
   }
+}
+
+int topk_sample_rows(const float* vals, const int32_t* idx, int64_t rows, int k, float temperature,
+                     const float* u, int32_t* token, void* stream) {
+  if (!vals || !idx || !u || !token) return TOPK_EINVAL;
+  if (rows < 1 || k < 1) return TOPK_EINVAL;
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(1.0f / temperature))
+    return TOPK_EINVAL;
+  if (k > kMaxK) return TOPK_EUNSUPPORTED;
+  const int64_t blocks = (rows + kSampleWarps - 1) / kSampleWarps;
+  if (blocks > 2147483647LL) return TOPK_EUNSUPPORTED;
+  int rc;
+  if ((rc = prepare_kernel(sample_rows_kernel))) return rc;
+  return launch_pdl(sample_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * kSampleWarps),
+                    0, static_cast<cudaStream_t>(stream), vals, idx, rows, k, 1.0f / temperature, u,
+                    token);
+}
+
+int topk_sample(const float* logits, int64_t rows, int64_t n, int k, int b, int kb,
+                float temperature, const float* u, int32_t* token, float* out_vals,
+                int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!u || !token) return TOPK_EINVAL;
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(1.0f / temperature))
+    return TOPK_EINVAL;
+  int rc = topk_bucketed(logits, rows, n, k, b, kb, out_vals, out_idx, workspace, workspace_bytes,
+                         stream);
+  if (rc) return rc;
+  return topk_sample_rows(out_vals, out_idx, rows, k, temperature, u, token, stream);
 }
 
 int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,

@@ -125,6 +125,33 @@ int topk_bucketed_merge(const float *vals_dev, const int32_t *idx_dev, int parts
                         int m, const int64_t *part_offset, int64_t n_total, int k, int b, int kb,
                         float *out_vals_dev, int32_t *out_idx_dev, void *stream);
 
+/* Sampling tail of top-k vocabulary sampling (the review page's "Core claim"
+ * and Fig. 4, left: vocabulary sampling keeps the top k of n logits).  The
+ * pages leave the tail implicit; this is plain top-k sampling.  For each row
+ * of selected pairs (best-first, as the selection calls write them), index
+ * idx[i] is drawn with probability w_i / sum_j w_j, w_i = exp((v_i - v_0)/T),
+ * by inverse CDF with the caller's uniform u[r] in [0, 1): the first i whose
+ * running sum of w exceeds u[r] * sum w (else, from rounding, the last entry
+ * of positive weight).  Padding (index -1) and -inf values weigh 0.  A row
+ * whose best value is NaN or +inf draws idx[0]; a row with no candidate
+ * draws -1.  Weights and sums are fp32.
+ *   vals_dev, idx_dev  [rows x k] selected values / indices (device).
+ *   temperature        T > 0 with 1/T finite (else TOPK_EINVAL).
+ *   u_dev              [rows] float32 uniforms in [0, 1), supplied by the
+ *                      caller (the library draws no random numbers).
+ *   token_dev          [rows] int32 output.
+ * No workspace.  Asynchronous on `stream`. */
+int topk_sample_rows(const float *vals_dev, const int32_t *idx_dev, int64_t rows, int k,
+                     float temperature, const float *u_dev, int32_t *token_dev, void *stream);
+
+/* topk_bucketed followed by topk_sample_rows on its output: the selection
+ * and the sampling tail of vocabulary sampling in two kernels on `stream`
+ * (the second starts as the first drains).  Arguments as in those two calls;
+ * out_vals_dev / out_idx_dev receive the selection. */
+int topk_sample(const float *logits_dev, int64_t rows, int64_t n, int k, int b, int kb,
+                float temperature, const float *u_dev, int32_t *token_dev, float *out_vals_dev,
+                int32_t *out_idx_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
+
 /* Fused selector: score[r][i] = sum_t q[r][t] * K_r[i][t] (bf16 inputs, fp32
  * accumulation; no 1/sqrt(d) scaling), then topk_bucketed on each row of
  * scores -- the sparse-attention selector that scores the current query

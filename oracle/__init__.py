@@ -75,9 +75,11 @@ class Oracle:
         lib.oracle_bucketed_pairs.argtypes = [p, p, i64, i64, i64, i64, p, p]
         lib.oracle_scores.argtypes = [p, i64, i64, p, i64, i64, p]
         lib.oracle_score_topk.argtypes = [p, i64, i64, p, i64, i64, i64, i64, i64, p, p, p]
+        lib.oracle_sample_row.argtypes = [p, p, i64, ctypes.c_double, ctypes.c_double, p, p]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         for f in ("oracle_bucketed", "oracle_exact", "oracle_bucketed_pairs", "oracle_scores",
-                  "oracle_score_topk", "oracle_get_threads", "oracle_max_threads"):
+                  "oracle_score_topk", "oracle_sample_row", "oracle_get_threads",
+                  "oracle_max_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.path = libpath
@@ -129,6 +131,24 @@ class Oracle:
         if rc:
             raise ValueError("oracle_bucketed_pairs failed (%d)" % rc)
         return ov, oi
+
+    def sample_rows(self, values, indices, temperature: float, u):
+        """Top-k sampling tail per row: (tokens [rows] int32, margins [rows])."""
+        v = np.ascontiguousarray(np.atleast_2d(np.asarray(values, np.float32)))
+        i = np.ascontiguousarray(np.atleast_2d(np.asarray(indices, np.int32)))
+        uu = np.asarray(u, np.float64).ravel()
+        rows, k = v.shape
+        tok = np.empty(rows, np.int32)
+        mar = np.empty(rows, np.float64)
+        one_t = ctypes.c_int32()
+        one_m = ctypes.c_double()
+        for r in range(rows):
+            rc = self.lib.oracle_sample_row(_ptr(v[r]), _ptr(i[r]), k, 1.0 / float(temperature),
+                                            float(uu[r]), ctypes.byref(one_t), ctypes.byref(one_m))
+            if rc:
+                raise ValueError("oracle_sample_row failed (%d)" % rc)
+            tok[r], mar[r] = one_t.value, one_m.value
+        return tok, mar
 
     def scores(self, q_bits, K_bits, kstride: int | None = None):
         """fp64-accumulated scores q . K_i rounded to float32.
@@ -226,6 +246,10 @@ def bucketed_pairs(values, indices, k, b, kb):
 
 def scores(q_bits, K_bits, kstride=None):
     return default().scores(q_bits, K_bits, kstride)
+
+
+def sample_rows(values, indices, temperature, u):
+    return default().sample_rows(values, indices, temperature, u)
 
 
 def score_topk(q_bits, K_bits, k, b, kb):

@@ -225,6 +225,54 @@ int oracle_bucketed_pairs(const float *v, const int32_t *idx, int64_t m, int64_t
     return 0;
 }
 
+/* Sampling tail of vocabulary sampling (the review page's "Core claim":
+ * top-k vocabulary sampling with n = 128,256 and k = 256 is one of the three
+ * workloads; Fig. 4, left).  The pages do not write the tail out; this is the
+ * plain reading of top-k sampling.  From the selected (value, index) pairs of
+ * one row, best-first, index idx[i] is drawn with probability
+ *     w_i / sum_j w_j,   w_i = exp((v_i - v_0) / T),
+ * by inverse CDF with the caller's uniform u in [0, 1): the first i whose
+ * running sum of w exceeds u * sum w (the last positive-weight entry if
+ * rounding leaves none).  Padding (index -1) and -inf values weigh 0.  When
+ * v_0 is NaN or +inf the draw is idx[0]; with no candidate it is -1.  All in
+ * double.  *margin receives min_i |running_sum_i - u * sum| / sum, the
+ * relative distance of the draw from its nearest CDF boundary. */
+int oracle_sample_row(const float *v, const int32_t *idx, int64_t k, double inv_t, double u,
+                      int32_t *token, double *margin)
+{
+    *margin = INFINITY;
+    if (k < 1 || idx[0] < 0) {
+        *token = -1;
+        return 0;
+    }
+    if (isnan(v[0]) || (isinf(v[0]) && v[0] > 0)) {
+        *token = idx[0];
+        return 0;
+    }
+    double total = 0.0;
+    for (int64_t i = 0; i < k; ++i)
+        if (idx[i] >= 0)
+            total += exp(((double)v[i] - (double)v[0]) * inv_t);
+    const double target = u * total;
+    double run = 0.0;
+    int32_t pick = -1, last = -1;
+    for (int64_t i = 0; i < k; ++i) {
+        if (idx[i] < 0)
+            continue;
+        const double w = exp(((double)v[i] - (double)v[0]) * inv_t);
+        if (w > 0.0)
+            last = idx[i];
+        run += w;
+        const double gap = fabs(run - target) / total;
+        if (gap < *margin)
+            *margin = gap;
+        if (pick < 0 && run > target)
+            pick = idx[i];
+    }
+    *token = pick >= 0 ? pick : last;
+    return 0;
+}
+
 static double bf16_to_double(uint16_t h)
 {
     uint32_t u = (uint32_t)h << 16;

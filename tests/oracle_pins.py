@@ -338,3 +338,62 @@ ALL_PINS = [
     pin_adversarial, pin_split_merge, pin_scores_unit_vectors, pin_scores_closed_form,
     pin_scores_numpy_fp64, pin_score_topk_selects_scores,
 ]
+
+
+# ---------------------------------------------------------------- sampling tail
+def pin_sampling_closed_forms(orc):
+    """Inverse-CDF draws at hand-computed boundaries."""
+    # two equal logits: the CDF boundary sits at exactly 1/2 (strictly above
+    # the target picks), so u < 1/2 draws the first and u >= 1/2 the second
+    v = np.array([[1.5, 1.5]], np.float32)
+    i = np.array([[7, 3]], np.int32)
+    for u, want in ((0.0, 7), (0.25, 7), (0.4999, 7), (0.5, 3), (0.75, 3), (0.9999, 3)):
+        t, _ = orc.sample_rows(v, i, 1.0, [u])
+        assert t[0] == want, (u, t[0], want)
+    # logits ln 3, 0 at T = 1: probabilities 3/4, 1/4
+    v = np.array([[math.log(3.0), 0.0]], np.float32)
+    i = np.array([[0, 1]], np.int32)
+    for u, want in ((0.74, 0), (0.76, 1)):
+        assert orc.sample_rows(v, i, 1.0, [u])[0][0] == want
+    # the same logits at T = 2 weigh sqrt(3) : 1, boundary sqrt(3)/(sqrt(3)+1) = 0.634
+    for u, want in ((0.62, 0), (0.65, 1)):
+        assert orc.sample_rows(v, i, 2.0, [u])[0][0] == want
+    # at T = 1/2 they weigh 9 : 1, boundary 0.9
+    for u, want in ((0.89, 0), (0.91, 1)):
+        assert orc.sample_rows(v, i, 0.5, [u])[0][0] == want
+
+
+def pin_sampling_frequencies(orc, N: int = 4000, seed: int = 11):
+    """Stratified uniforms u_j = (j + 1/2) / N: each token is drawn
+    round(N p_i) times up to one, p = softmax(v / T) over the selection."""
+    g = np.random.default_rng(seed)
+    for T in (0.5, 1.0, 3.0):
+        k = 12
+        v = np.sort(g.normal(size=k).astype(np.float32))[::-1].copy()
+        idx = g.permutation(1000)[:k].astype(np.int32)
+        rows_v = np.repeat(v[None], N, 0)
+        rows_i = np.repeat(idx[None], N, 0)
+        u = (np.arange(N) + 0.5) / N
+        tok, _ = orc.sample_rows(rows_v, rows_i, T, u)
+        p = np.exp((v.astype(np.float64) - v[0]) / T)
+        p /= p.sum()
+        for j in range(k):
+            assert abs(int((tok == idx[j]).sum()) - N * p[j]) <= 1.0 + 1e-9, (T, j)
+
+
+def pin_sampling_special(orc):
+    """Padding and -inf weigh nothing; a NaN or +inf best entry is drawn;
+    a row without candidates draws -1."""
+    ninf = -np.inf
+    v = np.array([[2.0, ninf, ninf], [np.nan, 1.0, 0.0], [np.inf, 5.0, 1.0], [ninf, ninf, ninf]],
+                 np.float32)
+    i = np.array([[4, 8, -1], [6, 2, 1], [9, 3, 0], [-1, -1, -1]], np.int32)
+    for u in (0.0, 0.5, 0.999):
+        t, _ = orc.sample_rows(v, i, 1.0, [u] * 4)
+        assert list(t) == [4, 6, 9, -1], (u, list(t))
+    # a padding slot in the middle of a list (whatever value it carries) moves
+    # no boundary: three equal weights, boundaries at 1/3 and 2/3
+    v = np.array([[1.0, 1.0, 1.0, 1.0]], np.float32)
+    i = np.array([[1, -1, 2, 3]], np.int32)
+    for u, want in ((0.3, 1), (0.6, 2), (0.9, 3)):
+        assert orc.sample_rows(v, i, 1.0, [u])[0][0] == want, u

@@ -98,6 +98,21 @@ def test_merge_rejects_bad_arguments_on_host(lib):
     assert call(k=20000) == U
 
 
+def test_sampling_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    E = atk.TOPK_EINVAL
+    assert lib.topk_sample_rows(None, p, 1, 4, 1.0, p, p, None) == E
+    assert lib.topk_sample_rows(p, p, 1, 4, 1.0, None, p, None) == E
+    assert lib.topk_sample_rows(p, p, 1, 4, 1.0, p, None, None) == E
+    assert lib.topk_sample_rows(p, p, 0, 4, 1.0, p, p, None) == E
+    assert lib.topk_sample_rows(p, p, 1, 0, 1.0, p, p, None) == E
+    for t in (0.0, -1.0, float("inf"), float("nan"), 1e-45):
+        assert lib.topk_sample_rows(p, p, 1, 4, t, p, p, None) == E, t
+        assert lib.topk_sample(p, 1, 8, 4, 2, 1, t, p, p, p, p, None, 0, None) == E, t
+    assert lib.topk_sample(p, 1, 8, 4, 2, 1, 1.0, None, p, p, p, None, 0, None) == E
+    assert lib.topk_sample(None, 1, 8, 4, 2, 1, 1.0, p, p, p, p, None, 0, None) == E
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
 

@@ -47,6 +47,22 @@ MUTANTS = [
      "const uint16_t *Kr = K + r * kstride;",
      "const uint16_t *Kr = K + 0 * kstride;",
      [P.pin_scores_unit_vectors, P.pin_scores_numpy_fp64]),
+    ("sampling weights with the sign of the exponent flipped",
+     "total += exp(((double)v[i] - (double)v[0]) * inv_t);",
+     "total += exp(((double)v[0] - (double)v[i]) * inv_t);",
+     [P.pin_sampling_closed_forms, P.pin_sampling_frequencies]),
+    ("sampling boundary taken inclusively",
+     "if (pick < 0 && run > target)",
+     "if (pick < 0 && run >= target)",
+     [P.pin_sampling_closed_forms]),
+    ("temperature multiplied instead of divided",
+     "const double w = exp(((double)v[i] - (double)v[0]) * inv_t);",
+     "const double w = exp(((double)v[i] - (double)v[0]) / inv_t);",
+     [P.pin_sampling_closed_forms, P.pin_sampling_frequencies]),
+    ("padding entries given weight",
+     "        if (idx[i] < 0)\n            continue;\n        const double w",
+     "        const double w",
+     [P.pin_sampling_special]),
 ]
 
 

@@ -65,3 +65,15 @@ def test_padding_when_few_candidates(oracle_mod):
     assert c[0] == 3
     assert list(i[0]) == [9, 8, 7, -1, -1, -1, -1, -1]
     assert np.all(np.isneginf(v[0, 3:]))
+
+
+def test_sampling_closed_forms(oracle_mod):
+    P.pin_sampling_closed_forms(oracle_mod.default())
+
+
+def test_sampling_frequencies(oracle_mod):
+    P.pin_sampling_frequencies(oracle_mod.default())
+
+
+def test_sampling_special(oracle_mod):
+    P.pin_sampling_special(oracle_mod.default())
