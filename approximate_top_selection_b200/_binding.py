@@ -61,6 +61,8 @@ def load_library():
             lib.topk_bucketed_merge.argtypes = [p, p, i32, i64, i32, ctypes.POINTER(ctypes.c_int64),
                                                 i64, i32, i32, i32, p, p, p]
             lib.topk_bucketed_merge.restype = i32
+            lib.score_rerank.argtypes = [p, i64, i32, p, i64, i64, p, i32, i32, p, p, p, p]
+            lib.score_rerank.restype = i32
             f32 = ctypes.c_float
             lib.topk_sample_rows.argtypes = [p, p, i64, i32, f32, p, p, p]
             lib.topk_sample_rows.restype = i32
@@ -254,6 +256,40 @@ def topk_bucketed_merge(vals: torch.Tensor, idx: torch.Tensor, n_total: int, k: 
                                      n_total, k, b, kb, out_vals.data_ptr(), out_idx.data_ptr(), sh)
     _check(st, "topk_bucketed_merge")
     return out_vals, out_idx
+
+
+def score_rerank(q: torch.Tensor, K: torch.Tensor, cand_idx: torch.Tensor, k: int, *,
+                 return_scores: bool = False, out_vals=None, out_idx=None, stream=None):
+    """Exact scores of each row's distinct candidate indices and their top-k.
+
+    q: [rows, d] bf16; K: [rows, n, d] or [n, d] bf16; cand_idx: [rows, c]
+    int32 (-1 = empty).  Returns (values, indices[, per-slot scores]).
+    """
+    lib = load_library()
+    _cuda(q, "q", torch.bfloat16)
+    _cuda(K, "K", torch.bfloat16)
+    _cuda(cand_idx, "cand_idx", torch.int32)
+    if q.dim() != 2 or cand_idx.dim() != 2 or cand_idx.shape[0] != q.shape[0]:
+        raise ValueError("q must be [rows, d] and cand_idx [rows, c]")
+    rows, d = q.shape
+    c = cand_idx.shape[1]
+    if K.dim() == 3:
+        if K.shape[0] != rows or K.shape[2] != d:
+            raise ValueError("K must be [rows, n, d] or [n, d]")
+        n, kstride = K.shape[1], K.shape[1] * d
+    elif K.dim() == 2 and K.shape[1] == d:
+        n, kstride = K.shape[0], 0
+    else:
+        raise ValueError("K must be [rows, n, d] or [n, d]")
+    with torch.cuda.device(q.device):
+        sh = _stream_handle(stream)
+        out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
+        scores = torch.empty(rows, c, dtype=torch.float32, device=q.device) if return_scores else None
+        st = lib.score_rerank(q.data_ptr(), rows, d, K.data_ptr(), n, kstride, cand_idx.data_ptr(), c,
+                              k, out_vals.data_ptr(), out_idx.data_ptr(),
+                              scores.data_ptr() if scores is not None else None, sh)
+    _check(st, "score_rerank")
+    return (out_vals, out_idx, scores) if return_scores else (out_vals, out_idx)
 
 
 def topk_sample_rows(vals: torch.Tensor, idx: torch.Tensor, temperature: float, u: torch.Tensor, *,

@@ -56,6 +56,7 @@ struct SelectArgs {
   T* out_vals;
   int32_t* out_idx;
   RowSplit rs;
+  SampleTail tail;  // token == nullptr: no sampling tail
 };
 
 // Shared-memory layout of the selection kernels (bytes).
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     }
     group_sync(kThreads);
     finish_piece<KB, kGatherInput, T>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
-                                      p.x + row0, p.out_vals, p.out_idx, piece_flag, nl);
+                                      p.x + row0, p.out_vals, p.out_idx, piece_flag, nl, p.tail);
     group_sync(kThreads);
   }
 }
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs<T> 
       q.store(w, lanebuf + static_cast<size_t>(tid + kThreads * w) * KB);
     group_sync(kThreads);
     finish_piece<KB, kGatherInput, T>(rs, b, p.k, r, a, len, lanebuf, cand, p.x + row0, p.out_vals,
-                                      p.out_idx, &piece_flag);
+                                      p.out_idx, &piece_flag, kLanes, p.tail);
     group_sync(kThreads);
     g = pend;
   }

@@ -569,6 +569,81 @@ __device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xr
   finalize_row_fast<VS, V>(cand, C, k, xrow, ov, oi);
 }
 
+// ------------------------------------------------------------------ sampling tail
+// Top-k sampling of one row by one warp: from the k selected pairs (v, ix),
+// best-first, index ix[i] is drawn with probability w_i / sum w,
+// w_i = exp((v_i - v_0) * inv_t), by inverse CDF with the uniform u: the
+// first i whose running sum exceeds u * sum w, else (rounding) the last entry
+// of positive weight.  Padding (-1) and -inf weigh 0; a NaN or +inf best
+// entry is drawn outright; no candidate draws -1.  Each lane sums a contiguous
+// slice in fp32 and a shuffle scan gives it the weight before its slice.
+// v and ix are plain loads: they may have been written by this CTA.
+__device__ __forceinline__ void sample_row_warp(const float* v, const int32_t* ix, int k,
+                                                float inv_t, float u, int32_t* token) {
+  const int lane = threadIdx.x & 31;
+  const int32_t i0 = ix[0];
+  const float v0 = v[0];
+  if (i0 < 0 || v0 != v0 || v0 == __int_as_float(0x7f800000)) {
+    if (lane == 0) *token = i0;  // -1 (no candidate), or the NaN / +inf entry
+    return;
+  }
+  const int per = (k + 31) / 32;
+  const int beg = min(lane * per, k), end = min(beg + per, k);
+  float part = 0.0f;
+  for (int i = beg; i < end; ++i)
+    if (ix[i] >= 0) part += expf((v[i] - v0) * inv_t);
+  float incl = part;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const float total = __shfl_sync(0xffffffffu, incl, 31);
+  const float target = u * total;
+  float run = incl - part;
+  int32_t pick = -1, last = -1;
+  for (int i = beg; i < end; ++i) {
+    if (ix[i] < 0) continue;
+    const float w = expf((v[i] - v0) * inv_t);
+    if (w > 0.0f) last = ix[i];
+    run += w;
+    if (run > target) {
+      pick = ix[i];
+      break;
+    }
+  }
+  const unsigned picked = __ballot_sync(0xffffffffu, pick >= 0);
+  const unsigned lasted = __ballot_sync(0xffffffffu, last >= 0);
+  const int src = picked ? __ffs(picked) - 1 : (lasted ? 31 - __clz(lasted) : 0);
+  const int32_t t = __shfl_sync(0xffffffffu, picked ? pick : last, src);
+  if (lane == 0) *token = t;
+}
+
+// Optional sampling tail of a selection call (token == nullptr: none).
+struct SampleTail {
+  const float* u;  // [rows] uniforms
+  int32_t* token;  // [rows]
+  float inv_t;     // 1 / temperature
+};
+
+// Out of line so that the streaming loop of the selection kernels keeps its
+// registers: the draw runs once per row, after Stage 2.
+__device__ __noinline__ void sample_row_warp_call(const float* v, const int32_t* ix, int k,
+                                                  float inv_t, float u, int32_t* token) {
+  sample_row_warp(v, ix, k, inv_t, u, token);
+}
+
+// After Stage 2 of row r wrote ov / oi (and the CTA met at a barrier): warp 0
+// draws the row's token.  Float rows only.
+template <typename V>
+__device__ __forceinline__ void run_sample_tail(const SampleTail& tail, int64_t r, int k,
+                                                const V* ov, const int32_t* oi) {
+  if constexpr (sizeof(V) == 4) {
+    if (tail.token != nullptr && threadIdx.x < 32)
+      sample_row_warp_call(ov, oi, k, tail.inv_t, __ldg(tail.u + r), tail.token + r);
+  }
+}
+
 // ------------------------------------------------------------------ pieces
 struct RowSplit {
   int64_t rows, n;  // row length in elements (scores or keys)
@@ -590,7 +665,8 @@ __device__ __forceinline__ int64_t cta_start(const RowSplit& rs, int c) {
 template <int KB, ValueSource VS, typename V>
 __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_t a, int64_t len,
                              const uint64_t* lanebuf, uint64_t* cand, const V* xrow, V* out_vals,
-                             int32_t* out_idx, int* s_flag, int nl = kLanes) {
+                             int32_t* out_idx, int* s_flag, int nl = kLanes,
+                             const SampleTail& tail = SampleTail{nullptr, nullptr, 1.0f}) {
   constexpr int T = kThreads;
   const int C = b * KB;
   V* ov = out_vals + r * static_cast<int64_t>(k);
@@ -599,6 +675,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
     merge_lanes<KB>(lanebuf, b, 0, cand, T, nl);
     group_sync(T);
     stage2<VS, V>(cand, C, k, xrow, ov, oi);
+    run_sample_tail<V>(tail, r, k, ov, oi);
     return;
   }
   const int64_t row0 = r * rs.n;
@@ -638,6 +715,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
   }
   group_sync(T);
   stage2<VS, V>(cand, C, k, xrow, ov, oi);
+  run_sample_tail<V>(tail, r, k, ov, oi);
   if (threadIdx.x == 0) rs.tickets[r] = 0u;  // leave the workspace zeroed
 }
 

@@ -14,6 +14,7 @@
 #include "bucket_select.cuh"
 #include "exact_topk.cuh"
 #include "merge_select.cuh"
+#include "rerank.cuh"
 #include "sample.cuh"
 #include "score_gemv.cuh"
 #include "score_umma.cuh"
@@ -361,7 +362,8 @@ int launch_select(int kb, bool fast, const Plan& pl, const SelectArgs<T>& a, cud
 // topk_bucketed for either element type.
 template <typename T>
 int run_bucketed(const T* scores, int64_t rows, int64_t n, int k, int b, int kb, T* out_vals,
-                 int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream) {
+                 int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream,
+                 const SampleTail& tail = SampleTail{nullptr, nullptr, 1.0f}) {
   if (!scores || !out_vals || !out_idx) return TOPK_EINVAL;
   int rc = check_common(rows, n, k, b, kb);
   if (rc) return rc;
@@ -381,6 +383,7 @@ int run_bucketed(const T* scores, int64_t rows, int64_t n, int k, int b, int kb,
   a.out_vals = out_vals;
   a.out_idx = out_idx;
   a.rs = make_split(pl, rows, n, workspace);
+  a.tail = tail;
   return launch_select<T>(kb, fast, pl, a, static_cast<cudaStream_t>(stream));
 }
 
@@ -616,6 +619,7 @@ int topk_bucketed_noalloc(const float* scores, int64_t rows, int64_t n, int k, i
   a.out_vals = out_vals;
   a.out_idx = out_idx;
   a.rs = make_split(pl, rows, n, scratch);
+  a.tail = SampleTail{nullptr, nullptr, 1.0f};
   return launch_select<float>(kb, fast, pl, a, st);
 }
 
@@ -685,6 +689,30 @@ int topk_bucketed_merge(const float* vals, const int32_t* idx, int parts, int64_
   }
 }
 
+int score_rerank(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,
+                 int64_t k_batch_stride, const int32_t* cand_idx, int c, int k, float* out_vals,
+                 int32_t* out_idx, float* out_scores, void* stream) {
+  if (!q || !K || !cand_idx || !out_vals || !out_idx) return TOPK_EINVAL;
+  if (rows < 1 || n < 1 || n > kMaxN || c < 1 || k < 1 || k_batch_stride < 0) return TOPK_EINVAL;
+  if (d != 128 && d != 256) return TOPK_EUNSUPPORTED;
+  if (c > kRerankMaxC || k > kMaxK || rows > 2147483647LL) return TOPK_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(K) || (k_batch_stride % 8) != 0) return TOPK_EINVAL;
+  DeviceInfo dev;
+  int rc = current_device_info(&dev);
+  if (rc) return rc;
+  const size_t smem = stage2_bytes(c) + static_cast<size_t>(rerank_table_size(c)) * 4;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  RerankArgs a{q, K, cand_idx, rows, n, k_batch_stride, c, k, out_vals, out_idx, out_scores};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(static_cast<unsigned>(rows)), block(kThreads);
+  if (d == 128) {
+    if ((rc = prepare_kernel(rerank_kernel<128>))) return rc;
+    return launch_pdl(rerank_kernel<128>, grid, block, smem, st, a);
+  }
+  if ((rc = prepare_kernel(rerank_kernel<256>))) return rc;
+  return launch_pdl(rerank_kernel<256>, grid, block, smem, st, a);
+}
+
 int topk_sample_rows(const float* vals, const int32_t* idx, int64_t rows, int k, float temperature,
                      const float* u, int32_t* token, void* stream) {
   if (!vals || !idx || !u || !token) return TOPK_EINVAL;
@@ -707,10 +735,10 @@ int topk_sample(const float* logits, int64_t rows, int64_t n, int k, int b, int 
   if (!u || !token) return TOPK_EINVAL;
   if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(1.0f / temperature))
     return TOPK_EINVAL;
-  int rc = topk_bucketed(logits, rows, n, k, b, kb, out_vals, out_idx, workspace, workspace_bytes,
-                         stream);
-  if (rc) return rc;
-  return topk_sample_rows(out_vals, out_idx, rows, k, temperature, u, token, stream);
+  if (k > kMaxK) return TOPK_EUNSUPPORTED;
+  // The draw runs inside the selection kernel, right after each row's Stage 2.
+  return run_bucketed<float>(logits, rows, n, k, b, kb, out_vals, out_idx, workspace,
+                             workspace_bytes, stream, SampleTail{u, token, 1.0f / temperature});
 }
 
 int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,

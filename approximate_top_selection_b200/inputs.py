@@ -151,5 +151,21 @@ def link_inputs(queries: int, entities: int, d: int, seed: int, device="cpu"):
 
 
 # Seeds of the five workload families (one per family, fixed).
+def support_union(rows: int, n: int, supports: int, size: int, seed: int, device="cpu") -> torch.Tensor:
+    """rows x (supports * size) int32 candidate indices: the concatenation of
+    `supports` index sets of `size` positions of [0, n) per row, each a shifted
+    and partly redrawn copy of the first, so they overlap as the supports of
+    similar queries do ("Recall Before You Rank", abstract).  Repeats stay in."""
+    g = _gen(seed, "cpu")
+    first = torch.randint(0, n, (rows, size), generator=g)
+    parts = [first]
+    for s in range(1, supports):
+        p = torch.roll(first, shifts=7 * s, dims=1).clone()
+        redraw = torch.rand(rows, size, generator=g) < 0.3
+        p[redraw] = torch.randint(0, n, (int(redraw.sum()),), generator=g)
+        parts.append(p)
+    return torch.cat(parts, dim=1).to(torch.int32).to(device)
+
+
 SEEDS = {"tiny": 0x70B00000, "decode": 0x70B00001, "vocab": 0x70B00002, "link": 0x70B00003,
          "long": 0x70B00004}

@@ -40,7 +40,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "bucketed top-k GB/s of scores read vs HBM peak; rows/s; recall@k vs Eq.(1)"
 
-# name -> workload description.  kind: "score" (fused q.K + selection) or "select".
+# name -> workload description.  kind: "score" (fused q.K + selection), "select",
+# or "rerank" (exact scores of given candidate indices + top-k).
 CONFIGS = {
     "tiny": dict(kind="select", rows=8, n=4096, k=64, b=128, kb=1, dist="normal"),
     "decode": dict(kind="score", batch=16, heads=32, n=32768, d=128, k=512, b=256, kb=2),
@@ -49,11 +50,18 @@ CONFIGS = {
     # reduced cases profiled with ncu --set full (inputs still larger than L2)
     "decode-quarter": dict(kind="score", batch=4, heads=32, n=32768, d=128, k=512, b=256, kb=2),
     "link-quarter": dict(kind="score", queries=1024, n=1 << 18, d=256, k=100, b=1024, kb=1),
+    # exact re-ranking of reused supports against the decode key cache: per row
+    # the union of 4 overlapping supports of 512 keys, top-512 of their scores
+    "decode-rerank": dict(kind="rerank", batch=16, heads=32, n=32768, d=128, k=512, supports=4,
+                          support=512),
 }
 for _b in (128, 256, 512):
     for _kb in (1, 2, 4):
         CONFIGS["long-b%d-kb%d" % (_b, _kb)] = dict(kind="select", rows=256, n=131072, k=512,
                                                     b=_b, kb=_kb, dist="uniform")
+# vocabulary sampling with its tail: the selection, then one token per row drawn
+# from the softmax (T = 1) of the selected logits
+CONFIGS["vocab-sample"] = dict(CONFIGS["vocab"], sample=1.0)
 # bfloat16 score rows (the page's Fig. 10 repeats its configurations in bf16)
 for _name in ("vocab", "long-b128-kb1", "long-b256-kb2", "long-b512-kb4"):
     CONFIGS[_name + "-bf16"] = dict(CONFIGS[_name], dtype="bf16")
@@ -140,7 +148,16 @@ class Workload:
         self.name, self.cfg, self.device = name, CONFIGS[name], device
         c = self.cfg
         seed = inputs.SEEDS[name.split("-")[0]] + seed_offset
-        if c["kind"] == "score":
+        if c["kind"] == "rerank":
+            self.rows = c["batch"] * c["heads"]
+            self.q, self.K = inputs.decode_inputs(c["batch"], c["heads"], c["n"], c["d"], seed,
+                                                  device=device)
+            self.cand = inputs.support_union(self.rows, c["n"], c["supports"], c["support"],
+                                             seed ^ 0xCA, device=device)
+            distinct = sum(len(set(r.tolist())) for r in self.cand.cpu())
+            # the distinct key rows each query gathers, the queries, the candidate lists
+            self.in_bytes = distinct * c["d"] * 2 + self.q.numel() * 2 + self.cand.numel() * 4
+        elif c["kind"] == "score":
             if "batch" in c:
                 self.rows = c["batch"] * c["heads"]
                 self.q, self.K = inputs.decode_inputs(c["batch"], c["heads"], c["n"], c["d"], seed,
@@ -161,7 +178,13 @@ class Workload:
             if c.get("dtype") == "bf16":
                 self.x = self.x.to(torch.bfloat16)
             self.in_bytes = self.x.numel() * self.x.element_size()
-        self.out_bytes = self.rows * c["k"] * 8
+        # values (2 bytes for bf16 rows, else 4) + int32 indices
+        self.out_bytes = self.rows * c["k"] * (6 if c.get("dtype") == "bf16" else 8)
+        if c.get("sample"):
+            g = torch.Generator(device=device).manual_seed(seed ^ 0x5EED)
+            self.u = torch.rand(self.rows, generator=g, device=device, dtype=torch.float32)
+            self.in_bytes += self.rows * 4
+            self.out_bytes += self.rows * 4
         self.bytes = self.in_bytes + self.out_bytes
         self.larger_than_l2 = self.in_bytes > 126 * 2 ** 20
 
@@ -171,7 +194,34 @@ class Workload:
         c = self.cfg
         if c["kind"] == "score":
             return atk.score_topk(self.q, self.K, c["k"], c["b"], c["kb"], stream=stream)
+        if c["kind"] == "rerank":
+            return atk.score_rerank(self.q, self.K, self.cand, c["k"], stream=stream)
+        if c.get("sample"):
+            return atk.topk_sample(self.x, c["k"], c["b"], c["kb"], c["sample"], self.u, stream=stream)
         return atk.topk_bucketed(self.x, c["k"], c["b"], c["kb"], stream=stream)
+
+    def oracle_step(self, rows: int):
+        """A callable doing this workload's step with the oracle on its first `rows` rows."""
+        import oracle
+
+        c = self.cfg
+        if c["kind"] in ("score", "rerank"):
+            q = self.q[:rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+            K = (self.K[:rows] if self.K.dim() == 3 else self.K).cpu().contiguous().view(torch.int16)
+            K = K.numpy().view(np.uint16)
+            if c["kind"] == "rerank":
+                cand = self.cand[:rows].cpu().numpy()
+                return lambda: oracle.rerank(q, K, cand, c["k"])
+            return lambda: oracle.score_topk(q, K, c["k"], c["b"], c["kb"])
+        x = self.x[:rows].float().cpu().numpy()
+        if c.get("sample"):
+            u = self.u[:rows].cpu().numpy().astype(np.float64)
+
+            def run():
+                ov, oi = oracle.bucketed(x, c["k"], c["b"], c["kb"])
+                oracle.sample_rows(ov, oi, c["sample"], u)
+            return run
+        return lambda: oracle.bucketed(x, c["k"], c["b"], c["kb"])
 
     def describe(self):
         c = dict(self.cfg)
@@ -187,11 +237,14 @@ def _uses_tensor_cores(cfg) -> bool:
 def _kernel_name(cfg) -> str:
     if cfg["kind"] == "score":
         return "score_select_umma" if _uses_tensor_cores(cfg) else "score_select_gemv"
+    if cfg["kind"] == "rerank":
+        return "rerank_kernel"
     return "bucket_select_tma"
 
 
 def _launches_per_step(cfg) -> int:
-    return 2 if _uses_tensor_cores(cfg) else 1  # the tensor-core path adds a Stage-2 kernel
+    # the tensor-core path adds a Stage-2 kernel, sampling adds the draw
+    return 2 if _uses_tensor_cores(cfg) or cfg.get("sample") else 1
 
 
 def _rotations(w: Workload) -> int:
@@ -224,6 +277,13 @@ def exact_context(w: Workload, ms_bucketed: float, steps: int = 20):
         x = w.x.float() if w.x.dtype != torch.float32 else w.x
         out["exact_topk_ms"] = _time_ms(lambda: atk.topk_exact(x, c["k"]), steps)
         out["torch_topk_ms"] = _time_ms(lambda: torch.topk(w.x, c["k"], dim=1), steps)
+    elif c["kind"] == "rerank":
+        ci = w.cand.long().clamp_min(0)
+
+        def fn():  # gather the candidate keys, score them, top-k (repeats not removed)
+            kc = torch.gather(w.K, 1, ci[:, :, None].expand(-1, -1, w.K.shape[2]))
+            return torch.topk(torch.bmm(kc, w.q[:, :, None]).squeeze(-1).float(), c["k"], dim=1)
+        out["torch_gather_scores_topk_ms"] = _time_ms(fn, max(3, steps // 4))
     else:
         if w.K.dim() == 3:
             fn = lambda: torch.topk(torch.bmm(w.K, w.q[:, :, None]).squeeze(-1).float(),  # noqa: E731
@@ -243,6 +303,8 @@ def recall_report(w: Workload):
     from oracle import recall as rc
 
     c = w.cfg
+    if c["kind"] == "rerank":
+        return None  # exact on its candidates: nothing to compare with
     if c["kind"] == "score":
         rows = min(w.rows, 64)
         _, bi, s = atk.score_topk(w.q[:rows], w.K[:rows] if w.K.dim() == 3 else w.K, c["k"],
@@ -271,17 +333,9 @@ def cpu_baseline(w: Workload, budget_s: float = 10.0):
     c = w.cfg
 
     def run(rows):
+        step = w.oracle_step(rows)
         t0 = time.perf_counter()
-        if c["kind"] == "score":
-            q = w.q[:rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-            K = (w.K[:rows] if w.K.dim() == 3 else w.K).cpu().contiguous().view(torch.int16)
-            K = K.numpy().view(np.uint16)
-            t0 = time.perf_counter()
-            oracle.score_topk(q, K, c["k"], c["b"], c["kb"])
-        else:
-            x = w.x[:rows].cpu().numpy()
-            t0 = time.perf_counter()
-            oracle.bucketed(x, c["k"], c["b"], c["kb"])
+        step()
         return time.perf_counter() - t0
 
     probe = min(w.rows, max(1, threads))
@@ -482,19 +536,31 @@ def e2e(w: Workload, args, world):
 
     c = w.cfg
     steps = max(1, min(args.steps, args.e2e_steps))
-    if c["kind"] == "score":
+    if c["kind"] in ("score", "rerank"):
         hq = torch.empty(w.q.shape, dtype=w.q.dtype, pin_memory=True)
         hK = torch.empty(w.K.shape, dtype=w.K.dtype, pin_memory=True)
         hq.copy_(w.q)
         hK.copy_(w.K)
         dq, dK = torch.empty_like(w.q), torch.empty_like(w.K)
         h2d = hq.numel() * 2 + hK.numel() * 2
+        if c["kind"] == "rerank":
+            hc = torch.empty(w.cand.shape, dtype=w.cand.dtype, pin_memory=True)
+            hc.copy_(w.cand)
+            dc = torch.empty_like(w.cand)
+            h2d += hc.numel() * 4
     else:
         hx = torch.empty(w.x.shape, dtype=w.x.dtype, pin_memory=True)
         hx.copy_(w.x)
         dx = torch.empty_like(w.x)
-        h2d = hx.numel() * 4
-    hv = torch.empty(w.rows, c["k"], dtype=torch.float32, pin_memory=True)
+        h2d = hx.numel() * hx.element_size()
+        if c.get("sample"):
+            hu = torch.empty(w.u.shape, dtype=w.u.dtype, pin_memory=True)
+            hu.copy_(w.u)
+            du = torch.empty_like(w.u)
+            ht = torch.empty(w.rows, dtype=torch.int32, pin_memory=True)
+            h2d += hu.numel() * 4
+    hv = torch.empty(w.rows, c["k"], dtype=torch.bfloat16 if c.get("dtype") == "bf16" else torch.float32,
+                     pin_memory=True)
     hi = torch.empty(w.rows, c["k"], dtype=torch.int32, pin_memory=True)
     stream = torch.cuda.current_stream()
 
@@ -503,6 +569,16 @@ def e2e(w: Workload, args, world):
             dq.copy_(hq, non_blocking=True)
             dK.copy_(hK, non_blocking=True)
             v, i = atk.score_topk(dq, dK, c["k"], c["b"], c["kb"])
+        elif c["kind"] == "rerank":
+            dq.copy_(hq, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            dc.copy_(hc, non_blocking=True)
+            v, i = atk.score_rerank(dq, dK, dc, c["k"])
+        elif c.get("sample"):
+            dx.copy_(hx, non_blocking=True)
+            du.copy_(hu, non_blocking=True)
+            t, v, i = atk.topk_sample(dx, c["k"], c["b"], c["kb"], c["sample"], du)
+            ht.copy_(t, non_blocking=True)
         else:
             dx.copy_(hx, non_blocking=True)
             v, i = atk.topk_bucketed(dx, c["k"], c["b"], c["kb"])
@@ -519,7 +595,7 @@ def e2e(w: Workload, args, world):
     barrier(world)
     ms = max_over_ranks(ev0.elapsed_time(ev1), world) / steps
     return {"value": w.bytes * world / (ms * 1e-3) / 1e9, "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": w.rows * c["k"] * 8,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": w.out_bytes,
             "ms_per_step": ms, "steps": steps}
 
 
@@ -536,14 +612,7 @@ def run_reference(args, world, rank, local):
     # sample size: about 1 s of oracle work per step
     probe = cpu_baseline(w, budget_s=1.0)
     rows = max(1, min(w.rows, int(probe["rows_per_s"] * 1.0)))
-    if c["kind"] == "score":
-        q = w.q[:rows].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
-        K = (w.K[:rows] if w.K.dim() == 3 else w.K).cpu().contiguous().view(torch.int16)
-        K = K.numpy().view(np.uint16)
-        step = lambda: oracle.score_topk(q, K, c["k"], c["b"], c["kb"])  # noqa: E731
-    else:
-        x = w.x[:rows].cpu().numpy()
-        step = lambda: oracle.bucketed(x, c["k"], c["b"], c["kb"])  # noqa: E731
+    step = w.oracle_step(rows)
     for _ in range(min(args.warmup, 3)):
         step()
     steps = max(1, min(args.steps, 20))

@@ -125,6 +125,26 @@ int topk_bucketed_merge(const float *vals_dev, const int32_t *idx_dev, int parts
                         int m, const int64_t *part_offset, int64_t n_total, int k, int b, int kb,
                         float *out_vals_dev, int32_t *out_idx_dev, void *stream);
 
+/* Exact re-ranking of a candidate index set ("Recall Before You Rank",
+ * abstract: the supports retrieved for similar earlier queries are reused as
+ * candidates and scored exactly against the current query before the top-K
+ * is kept).  For row r: score_i = sum_t q[r][t] * K_r[i][t] (bf16 inputs,
+ * fp32 accumulation, no 1/sqrt(d)) for every DISTINCT index 0 <= i < n among
+ * cand_idx[r][0..c); the k best (score, index) pairs under the total order
+ * above, best-first, padded with -inf / -1.
+ *   q_dev, K_dev, d, n, k_batch_stride  as in score_topk (d 128 or 256;
+ *                16-byte aligned; k_batch_stride a multiple of 8).
+ *   cand_idx_dev [rows x c] int32 candidate indices: -1 marks an empty slot,
+ *                repeats are scored once, an index >= n is skipped and sets
+ *                TOPK_DEV_BAD_INDEX.  1 <= c <= 4096 (else TOPK_EUNSUPPORTED).
+ *   out_scores_dev  nullable [rows x c] float32: the fp32 score of each slot
+ *                (-inf for empty, repeated or skipped slots), for checking.
+ * Values are the fp32 scores (zero as +0.0, NaN as 0x7FFFFFFF).  No
+ * workspace.  Asynchronous on `stream`. */
+int score_rerank(const uint16_t *q_dev, int64_t rows, int d, const uint16_t *K_dev, int64_t n,
+                 int64_t k_batch_stride, const int32_t *cand_idx_dev, int c, int k,
+                 float *out_vals_dev, int32_t *out_idx_dev, float *out_scores_dev, void *stream);
+
 /* Sampling tail of top-k vocabulary sampling (the review page's "Core claim"
  * and Fig. 4, left: vocabulary sampling keeps the top k of n logits).  The
  * pages leave the tail implicit; this is plain top-k sampling.  For each row
@@ -144,10 +164,11 @@ int topk_bucketed_merge(const float *vals_dev, const int32_t *idx_dev, int parts
 int topk_sample_rows(const float *vals_dev, const int32_t *idx_dev, int64_t rows, int k,
                      float temperature, const float *u_dev, int32_t *token_dev, void *stream);
 
-/* topk_bucketed followed by topk_sample_rows on its output: the selection
- * and the sampling tail of vocabulary sampling in two kernels on `stream`
- * (the second starts as the first drains).  Arguments as in those two calls;
- * out_vals_dev / out_idx_dev receive the selection. */
+/* topk_bucketed with the draw of topk_sample_rows fused into it: the CTA
+ * that finishes a row's selection draws that row's token right away, so the
+ * selection and the sampling tail of vocabulary sampling take one kernel.
+ * Arguments as in those two calls (float32 logits); out_vals_dev /
+ * out_idx_dev receive the selection, token_dev the draws. */
 int topk_sample(const float *logits_dev, int64_t rows, int64_t n, int k, int b, int kb,
                 float temperature, const float *u_dev, int32_t *token_dev, float *out_vals_dev,
                 int32_t *out_idx_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
@@ -212,7 +233,7 @@ const char *topk_status_string(int status);
 int topk_device_status(int *status_out);
 
 #define TOPK_DEV_WAIT_TIMEOUT 1 /* a bulk-copy wait in a streaming kernel expired */
-#define TOPK_DEV_BAD_INDEX 2    /* topk_bucketed_merge skipped a pair with index >= n_total */
+#define TOPK_DEV_BAD_INDEX 2    /* topk_bucketed_merge or score_rerank skipped an index out of range */
 
 #ifdef __cplusplus
 }

@@ -75,10 +75,11 @@ class Oracle:
         lib.oracle_bucketed_pairs.argtypes = [p, p, i64, i64, i64, i64, p, p]
         lib.oracle_scores.argtypes = [p, i64, i64, p, i64, i64, p]
         lib.oracle_score_topk.argtypes = [p, i64, i64, p, i64, i64, i64, i64, i64, p, p, p]
+        lib.oracle_rerank.argtypes = [p, i64, i64, p, i64, i64, p, i64, i64, p, p]
         lib.oracle_sample_row.argtypes = [p, p, i64, ctypes.c_double, ctypes.c_double, p, p]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         for f in ("oracle_bucketed", "oracle_exact", "oracle_bucketed_pairs", "oracle_scores",
-                  "oracle_score_topk", "oracle_sample_row", "oracle_get_threads",
+                  "oracle_score_topk", "oracle_sample_row", "oracle_rerank", "oracle_get_threads",
                   "oracle_max_threads"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
@@ -130,6 +131,29 @@ class Oracle:
                                             _ptr(oi))
         if rc:
             raise ValueError("oracle_bucketed_pairs failed (%d)" % rc)
+        return ov, oi
+
+    def rerank(self, q_bits, K_bits, cand, k: int):
+        """Exact scores of each row's distinct candidate indices and their top-k.
+
+        q_bits [rows, d], K_bits [rows, n, d] or [n, d] (bf16 bit patterns),
+        cand [rows, c] int32 (-1 = empty).  Returns (values, indices) [rows, k].
+        """
+        q = _bf16_bits(q_bits)
+        K = _bf16_bits(K_bits)
+        rows, d = q.shape
+        if K.ndim == 2:
+            n, stride = K.shape[0], 0
+        else:
+            n, stride = K.shape[1], K.shape[1] * d
+        cidx = np.ascontiguousarray(np.asarray(cand, np.int32))
+        c = cidx.shape[1]
+        ov = np.empty((rows, k), np.float32)
+        oi = np.empty((rows, k), np.int32)
+        rc = self.lib.oracle_rerank(_ptr(q), rows, d, _ptr(K), n, stride, _ptr(cidx), c, k,
+                                    _ptr(ov), _ptr(oi))
+        if rc:
+            raise ValueError("oracle_rerank failed (%d)" % rc)
         return ov, oi
 
     def sample_rows(self, values, indices, temperature: float, u):
@@ -250,6 +274,10 @@ def scores(q_bits, K_bits, kstride=None):
 
 def sample_rows(values, indices, temperature, u):
     return default().sample_rows(values, indices, temperature, u)
+
+
+def rerank(q_bits, K_bits, cand, k):
+    return default().rerank(q_bits, K_bits, cand, k)
 
 
 def score_topk(q_bits, K_bits, k, b, kb):

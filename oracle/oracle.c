@@ -302,6 +302,59 @@ int oracle_scores(const uint16_t *q, int64_t rows, int64_t d, const uint16_t *K,
     return 0;
 }
 
+/* Re-ranking of a candidate index set ("Recall Before You Rank", abstract:
+ * the supports of similar earlier queries are reused as candidates and
+ * scored exactly against the current query before the top-K is kept).  Per
+ * row r: the distinct indices 0 <= i < n among cand[r][0..c) (-1 marks an
+ * empty slot; repeats and out-of-range indices are dropped), each scored as
+ * in oracle_scores, and the k best (score, index) pairs under the total
+ * order, best-first, padded with -inf / -1. */
+int oracle_rerank(const uint16_t *q, int64_t rows, int64_t d, const uint16_t *K, int64_t n,
+                  int64_t kstride, const int32_t *cand, int64_t c, int64_t k, float *out_vals,
+                  int32_t *out_idx)
+{
+    if (rows < 0 || d < 1 || n < 1 || c < 1 || k < 1 || kstride < 0)
+        return 1;
+    int fail = 0;
+#pragma omp parallel num_threads(g_threads)
+    {
+        item *all = (item *)malloc(sizeof(item) * (size_t)c);
+        if (!all) {
+#pragma omp atomic write
+            fail = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!all)
+                continue;
+            const uint16_t *qr = q + r * d;
+            const uint16_t *Kr = K + kstride * r; /* this row's key matrix */
+            const int32_t *cr = cand + r * c;
+            int64_t m = 0;
+            for (int64_t j = 0; j < c; ++j) {
+                const int64_t i = cr[j];
+                if (i < 0 || i >= n)
+                    continue;
+                int seen = 0;
+                for (int64_t t = 0; t < m && !seen; ++t)
+                    seen = all[t].i == i;
+                if (seen)
+                    continue;
+                double acc = 0.0; /* exact bf16 products, summed over t in order */
+                for (int64_t t = 0; t < d; ++t)
+                    acc += bf16_to_double(Kr[i * d + t]) * bf16_to_double(qr[t]);
+                all[m].v = (float)acc;
+                all[m].i = i;
+                ++m;
+            }
+            qsort(all, (size_t)m, sizeof(item), cmp_items);
+            write_row(all, m < k ? m : k, k, out_vals + r * k, out_idx + r * k);
+        }
+        free(all);
+    }
+    return fail ? 2 : 0;
+}
+
 /* Fused scoring then bucketed selection on the float scores. out_scores
  * (nullable) receives the rows*n float scores. */
 int oracle_score_topk(const uint16_t *q, int64_t rows, int64_t d, const uint16_t *K, int64_t n,

@@ -397,3 +397,43 @@ def pin_sampling_special(orc):
     i = np.array([[1, -1, 2, 3]], np.int32)
     for u, want in ((0.3, 1), (0.6, 2), (0.9, 3)):
         assert orc.sample_rows(v, i, 1.0, [u])[0][0] == want, u
+
+
+# ---------------------------------------------------------------- re-ranking
+def _bf16_bits(x: torch.Tensor) -> np.ndarray:
+    return x.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def pin_rerank_numpy(orc, seed: int = 12):
+    """Re-ranking = numpy fp64 scores of the distinct valid candidates (rounded
+    to float) + a lexsort top-k; repeats, -1 and out-of-range slots drop out."""
+    g = np.random.default_rng(seed)
+    rows, n, d, c, k = 5, 300, 128, 90, 20
+    q = torch.from_numpy(g.normal(size=(rows, d)).astype(np.float32))
+    K = torch.from_numpy((g.normal(size=(rows, n, d)) / np.sqrt(d)).astype(np.float32))
+    qb, Kb = _bf16_bits(q), _bf16_bits(K)
+    cand = g.integers(0, n, size=(rows, c)).astype(np.int32)  # repeats on purpose
+    cand[:, ::7] = -1
+    cand[:, 3] = n + 5  # out of range
+    ov, oi = orc.rerank(qb, Kb, cand, k)
+    qf = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    Kf = (Kb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for r in range(rows):
+        ids = np.array(sorted({int(i) for i in cand[r] if 0 <= i < n}), np.int64)
+        s = (Kf[r, ids] @ qf[r]).astype(np.float32)
+        order = np.lexsort((ids, -s.astype(np.float64)))[:k]
+        assert list(oi[r, :len(order)]) == list(ids[order]), r
+        assert np.array_equal(ov[r, :len(order)], s[order])
+        assert np.all(oi[r, len(order):] == -1)
+
+
+def pin_rerank_shared_keys_and_padding(orc):
+    """A key matrix shared by all rows; fewer distinct candidates than k pads."""
+    d, n = 128, 16
+    K = torch.zeros(n, d)
+    K[torch.arange(n), torch.arange(n)] = torch.arange(n, dtype=torch.float32)  # key i scores i*q_i
+    q = torch.ones(2, d)
+    cand = np.array([[3, 3, 9, -1, 1], [15, 0, 15, 15, 15]], np.int32)
+    ov, oi = orc.rerank(_bf16_bits(q), _bf16_bits(K), cand, 4)
+    assert list(oi[0]) == [9, 3, 1, -1] and list(ov[0, :3]) == [9.0, 3.0, 1.0]
+    assert list(oi[1]) == [15, 0, -1, -1] and list(ov[1, :2]) == [15.0, 0.0]

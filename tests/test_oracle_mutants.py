@@ -63,6 +63,14 @@ MUTANTS = [
      "        if (idx[i] < 0)\n            continue;\n        const double w",
      "        const double w",
      [P.pin_sampling_special]),
+    ("re-ranking keeps repeated candidates",
+     "                if (seen)\n                    continue;\n",
+     "",
+     [P.pin_rerank_numpy, P.pin_rerank_shared_keys_and_padding]),
+    ("re-ranking drops the last candidate slot",
+     "            for (int64_t j = 0; j < c; ++j) {\n                const int64_t i = cr[j];",
+     "            for (int64_t j = 0; j < c - 1; ++j) {\n                const int64_t i = cr[j];",
+     [P.pin_rerank_numpy, P.pin_rerank_shared_keys_and_padding]),
 ]
 
 

@@ -77,3 +77,11 @@ def test_sampling_frequencies(oracle_mod):
 
 def test_sampling_special(oracle_mod):
     P.pin_sampling_special(oracle_mod.default())
+
+
+def test_rerank_numpy(oracle_mod):
+    P.pin_rerank_numpy(oracle_mod.default())
+
+
+def test_rerank_shared_keys_and_padding(oracle_mod):
+    P.pin_rerank_shared_keys_and_padding(oracle_mod.default())
