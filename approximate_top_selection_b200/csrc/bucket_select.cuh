@@ -159,7 +159,9 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // the CTA's tiles into a ring of `stages` shared-memory stages (full barrier:
 // bytes landed; empty barrier: every consumer warp is done with the stage);
 // the kThreads consumer threads never wait for each other inside a piece.
-template <typename T, int KB>
+// SAMPLE: the instantiation that also draws each row's token after Stage 2
+// (p.tail); without it the sampling code is not compiled in at all.
+template <typename T, int KB, bool SAMPLE = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
                                                                   int cand_cap) {
   constexpr int kTileElems = Elem<T>::kPerTile;
@@ -312,7 +314,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     }
     group_sync(kThreads);
     finish_piece<KB, kGatherInput, T>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf, cand,
-                                      p.x + row0, p.out_vals, p.out_idx, piece_flag, nl, p.tail);
+                                      p.x + row0, p.out_vals, p.out_idx, piece_flag, nl,
+                                      SAMPLE ? p.tail : SampleTail{nullptr, nullptr, 1.0f});
     group_sync(kThreads);
   }
 }

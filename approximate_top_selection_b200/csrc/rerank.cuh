@@ -15,7 +15,8 @@
 // shared-memory hash set (first insert wins; duplicates carry identical
 // scores, so which copy survives does not matter).  A group of D/16 lanes
 // scores one candidate: each lane holds 16 query values in registers and
-// loads 16 key values with two 16-byte loads, and the group sums with
+// loads 16 key values with two 16-byte loads (two candidates in flight per
+// group; four CTAs per SM so that 512 rows fit one wave), and the group sums with
 // shuffles.  Scores become packed (order key, ~index) words, and the shared
 // Stage 2 keeps the top k.
 #pragma once
@@ -45,8 +46,15 @@ __host__ __device__ __forceinline__ int rerank_table_size(int c) {
   return h;
 }
 
+#ifndef TOPK_RERANK_INFLIGHT
+#define TOPK_RERANK_INFLIGHT 2
+#endif
+#ifndef TOPK_RERANK_MIN_CTAS
+#define TOPK_RERANK_MIN_CTAS 4
+#endif
+
 template <int D>
-__global__ void __launch_bounds__(kThreads) rerank_kernel(RerankArgs p) {
+__global__ void __launch_bounds__(kThreads, TOPK_RERANK_MIN_CTAS) rerank_kernel(RerankArgs p) {
   constexpr int G = D / 16;          // lanes per candidate
   constexpr int PER_WARP = 32 / G;   // candidates per warp per pass
   extern __shared__ __align__(128) unsigned char smem[];
@@ -104,7 +112,7 @@ __global__ void __launch_bounds__(kThreads) rerank_kernel(RerankArgs p) {
   const uint16_t* Kr = p.K + r * p.kstride;
   // R candidates per lane group in flight: their key loads are all issued
   // before any is used, so a warp keeps 2R 16-byte loads per lane outstanding.
-  constexpr int R = 4;
+  constexpr int R = TOPK_RERANK_INFLIGHT;
   constexpr int STEP = (kThreads / 32) * PER_WARP;  // candidates per CTA pass
   for (int base = warp * PER_WARP; base < C; base += R * STEP) {
     uint4 ka[R], kb[R];

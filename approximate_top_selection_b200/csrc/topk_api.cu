@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/topk_b200.h"
 #include "bucket_select.cuh"
@@ -342,6 +343,14 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 
 template <typename T, int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
+  if constexpr (std::is_same<T, float>::value) {
+    if (fast && a.tail.token != nullptr) {
+      int rc = prepare_kernel(bucket_select_tma<T, KB, true>);
+      if (rc) return rc;
+      return launch_pdl(bucket_select_tma<T, KB, true>, dim3(pl.G), dim3(kPipeThreads), pl.smem,
+                        st, a, pl.stages, pl.cand_cap);
+    }
+  }
   if (fast)
     return launch_pdl(bucket_select_tma<T, KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
                       pl.stages, pl.cand_cap);
