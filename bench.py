@@ -54,6 +54,8 @@ CONFIGS = {
     # the union of 4 overlapping supports of 512 keys, top-512 of their scores
     "decode-rerank": dict(kind="rerank", batch=16, heads=32, n=32768, d=128, k=512, supports=4,
                           support=512),
+    "decode-rerank-quarter": dict(kind="rerank", batch=4, heads=32, n=32768, d=128, k=512,
+                                  supports=4, support=512),
 }
 for _b in (128, 256, 512):
     for _kb in (1, 2, 4):
@@ -473,6 +475,7 @@ _KERNEL_SOURCES = {
     "bucket_select_tma": ("common.cuh", "select_core.cuh", "bucket_select.cuh"),
     "score_select_gemv": ("common.cuh", "select_core.cuh", "score_gemv.cuh"),
     "score_select_umma": ("common.cuh", "select_core.cuh", "score_umma.cuh"),
+    "rerank_kernel": ("common.cuh", "select_core.cuh", "rerank.cuh"),
 }
 
 
