@@ -85,10 +85,34 @@ def _check(status: int, where: str) -> None:
         raise TopkError(status, where)
 
 
-def _stream_handle(stream) -> int:
+def _stream_handle(stream, device_index: int) -> int:
+    """cudaStream_t of `stream`, or of the device's current stream."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        return torch._C._cuda_getCurrentRawStream(device_index)
     return int(stream.cuda_stream)
+
+
+class _OnDevice:
+    """Makes the tensor's device current for a call, switching only when it
+    is not current already (a device context costs microseconds per call)."""
+
+    __slots__ = ("index", "prev")
+
+    def __init__(self, device: torch.device):
+        self.index = device.index if device.index is not None else torch.cuda.current_device()
+        self.prev = None
+
+    def __enter__(self):
+        cur = torch.cuda.current_device()
+        if cur != self.index:
+            self.prev = cur
+            torch.cuda.set_device(self.index)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            torch.cuda.set_device(self.prev)
+        return False
 
 
 def _cuda(t: torch.Tensor, name: str, dtype) -> None:
@@ -157,8 +181,8 @@ def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=Non
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with torch.cuda.device(scores.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(scores.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         need = topk_workspace_bytes(TOPK_OP_BUCKETED, rows, n, k, b, kb)
         ws = workspace if workspace is not None else _workspace(need, scores.device, sh)
@@ -177,8 +201,8 @@ def topk_bucketed_bf16(scores: torch.Tensor, k: int, b: int, kb: int, *, out_val
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with torch.cuda.device(scores.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(scores.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx, torch.bfloat16)
         need = topk_workspace_bytes(TOPK_OP_BUCKETED_BF16, rows, n, k, b, kb)
         ws = workspace if workspace is not None else _workspace(need, scores.device, sh)
@@ -201,8 +225,8 @@ def topk_bucketed_noalloc(scores: torch.Tensor, k: int, b: int, kb: int, *, out_
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with torch.cuda.device(scores.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(scores.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         st = lib.topk_bucketed_noalloc(scores.data_ptr(), rows, n, k, b, kb, out_vals.data_ptr(),
                                        out_idx.data_ptr(), sh)
@@ -217,8 +241,8 @@ def topk_exact(scores: torch.Tensor, k: int, *, out_vals=None, out_idx=None, str
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with torch.cuda.device(scores.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(scores.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         st = lib.topk_exact(scores.data_ptr(), rows, n, k, out_vals.data_ptr(),
                             out_idx.data_ptr(), None, 0, sh)
@@ -249,8 +273,8 @@ def topk_bucketed_merge(vals: torch.Tensor, idx: torch.Tensor, n_total: int, k: 
     if len(offs) != parts:
         raise ValueError("part_offsets needs one entry per part")
     c_offs = (ctypes.c_int64 * parts)(*offs)
-    with torch.cuda.device(vals.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(vals.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, vals.device, out_vals, out_idx)
         st = lib.topk_bucketed_merge(vals.data_ptr(), idx.data_ptr(), parts, rows, m, c_offs,
                                      n_total, k, b, kb, out_vals.data_ptr(), out_idx.data_ptr(), sh)
@@ -281,8 +305,8 @@ def score_rerank(q: torch.Tensor, K: torch.Tensor, cand_idx: torch.Tensor, k: in
         n, kstride = K.shape[0], 0
     else:
         raise ValueError("K must be [rows, n, d] or [n, d]")
-    with torch.cuda.device(q.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(q.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
         scores = torch.empty(rows, c, dtype=torch.float32, device=q.device) if return_scores else None
         st = lib.score_rerank(q.data_ptr(), rows, d, K.data_ptr(), n, kstride, cand_idx.data_ptr(), c,
@@ -303,8 +327,8 @@ def topk_sample_rows(vals: torch.Tensor, idx: torch.Tensor, temperature: float, 
     if vals.dim() != 2 or tuple(idx.shape) != tuple(vals.shape) or u.numel() != vals.shape[0]:
         raise ValueError("vals, idx must be [rows, k] and u [rows]")
     rows, k = vals.shape
-    with torch.cuda.device(vals.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(vals.device) as on:
+        sh = _stream_handle(stream, on.index)
         if out_token is None:
             out_token = torch.empty(rows, dtype=torch.int32, device=vals.device)
         _cuda(out_token, "out_token", torch.int32)
@@ -324,8 +348,8 @@ def topk_sample(logits: torch.Tensor, k: int, b: int, kb: int, temperature: floa
     if logits.dim() != 2 or u.numel() != logits.shape[0]:
         raise ValueError("logits must be [rows, n] and u [rows]")
     rows, n = logits.shape
-    with torch.cuda.device(logits.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(logits.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, logits.device, out_vals, out_idx)
         if out_token is None:
             out_token = torch.empty(rows, dtype=torch.int32, device=logits.device)
@@ -364,8 +388,8 @@ def score_topk(q: torch.Tensor, K: torch.Tensor, k: int, b: int, kb: int, *,
         raise ValueError("K must be [rows, n, d] or [n, d]")
     if K.shape[-1] != d:
         raise ValueError("q and K disagree on d")
-    with torch.cuda.device(q.device):
-        sh = _stream_handle(stream)
+    with _OnDevice(q.device) as on:
+        sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
         scores = torch.empty(rows, n, dtype=torch.float32, device=q.device) if return_scores else None
         need = topk_workspace_bytes(TOPK_OP_SCORE, rows, n, k, b, kb, d)
