@@ -126,14 +126,25 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
       mask[u & 3] |=
           (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[u & 3]) ? (1u << u) : 0u;
   }
-  // Survivors of each queue in turn, re-read from shared memory.
+  // Survivors of each queue in turn, re-read from shared memory.  The loop is
+  // software-pipelined: the next survivor's value is loaded before the
+  // current one is inserted, so the load latency overlaps the insert.
   const T* tt = tile + t;
 #define TK_SURVIVORS(Q)                                                                   \
-  while (mask[Q]) {                                                                       \
-    const int u = __ffs(mask[Q]) - 1;                                                     \
+  if (mask[Q]) {                                                                          \
+    int u = __ffs(mask[Q]) - 1;                                                           \
     mask[Q] &= mask[Q] - 1u;                                                              \
-    q.template insert_fast<Q>(to_f32(tt[kThreads * u]),                                   \
-                              base + static_cast<uint32_t>(kThreads * u) - (Q));          \
+    float xc = to_f32(tt[kThreads * u]);                                                  \
+    for (;;) {                                                                            \
+      const bool more = mask[Q] != 0u;                                                    \
+      const int un = more ? __ffs(mask[Q]) - 1 : u;                                       \
+      const float xn = to_f32(tt[kThreads * un]);                                         \
+      q.template insert_fast<Q>(xc, base + static_cast<uint32_t>(kThreads * u) - (Q));    \
+      if (!more) break;                                                                   \
+      mask[Q] &= mask[Q] - 1u;                                                            \
+      u = un;                                                                             \
+      xc = xn;                                                                            \
+    }                                                                                     \
   }
   TK_SURVIVORS(0)
   if (nq > 1) {
