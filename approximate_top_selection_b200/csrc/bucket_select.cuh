@@ -1,20 +1,25 @@
-// bucket_select.cuh -- Stage 1 + Stage 2 of bucketed top-k over float32 rows.
+// bucket_select.cuh -- Stage 1 + Stage 2 of bucketed top-k over float32 or
+// bfloat16 score rows.
 //
 // Method: "Approximate Top-k for Increased Parallelism" (arXiv 2412.04358),
 // pith.science review page, "What carries the argument": interleaved buckets
 // (element i -> bucket i mod b), exact top-k_b per bucket kept in per-thread
 // register queues (k_b <= 4), final exact top-k when b*k_b > k.
 //
-// Work decomposition (ours, not the page's): the rows*n elements are cut into
-// G equal contiguous CTA ranges, so every CTA streams the same number of bytes
-// whatever the row count; a row that straddles CTA ranges is merged by the last
+// Work decomposition (ours, not the page's): one CTA per row when the rows
+// fill one resident wave, else the rows*n elements are cut into G equal
+// contiguous CTA ranges; a row that straddles CTA ranges is merged by the last
 // CTA to finish it (select_core.cuh).
 //
-// Fast kernel (n % 4 == 0, 16-byte aligned rows, b | 1024): the TMA engine
-// streams 16 KB tiles of the row into a ring of shared-memory stages
-// (cp.async.bulk + mbarrier); thread t owns the four consecutive positions
-// 4t..4t+3 of every 1024-element stripe, so each of its four queues sees a
-// single bucket ((a + 4t + v) mod b) and needs no communication until the end.
+// Fast kernel (n % 4 == 0 for fp32 / 8 for bf16, 16-byte aligned rows,
+// b | 1024): a producer warp streams 32 KB tiles of the row into a ring of
+// shared-memory stages (cp.async.bulk + mbarrier).  k_b <= 2: thread t owns
+// the four consecutive positions 4t..4t+3 of every 1024-element stripe, so
+// each of its four queues sees a single bucket ((a + 4t + v) mod b), updated
+// branch-free.  k_b > 2: queue q of thread t covers positions t + 256 q modulo
+// max(256, b); each element is tested against its queue's k_b-th value and
+// only survivors take the sorted insert.  An optional sampling tail (template
+// flag) draws one token per row after Stage 2.
 // General kernel (any n, alignment, b <= 1024): direct coalesced scalar loads,
 // thread t owns stripe positions t + 256 v of a stripe of L*b elements.
 #pragma once

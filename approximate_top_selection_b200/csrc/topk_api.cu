@@ -29,8 +29,9 @@ constexpr int64_t kMaxElems = 1LL << 50;      // keeps the partition arithmetic 
 constexpr int64_t kSelectMinPiece = 16384;    // elements per CTA before splitting pays
 constexpr int64_t kScoreMinPiece = 1024;      // keys per CTA
 
-// Ring depth: as many 16 KB stages as fit while kCtasPerSm CTAs share an SM's
-// shared memory (bytes in flight per SM are what keeps HBM busy), clamped.
+// Ring depth: as many tile stages (32 KB for score rows, 16 KB for key tiles)
+// as fit while kCtasPerSm CTAs share an SM's shared memory (bytes in flight
+// per SM are what keeps HBM busy), clamped.
 #ifndef TOPK_CTAS_PER_SM
 #define TOPK_CTAS_PER_SM 2
 #endif
