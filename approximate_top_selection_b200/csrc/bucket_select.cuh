@@ -336,6 +336,199 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
   }
 }
 
+// ------------------------------------------------------------------ k_b > 2, 16 warps
+// The k_b > 2 update is a chain of survivor inserts per queue, so it is bound
+// by latency rather than bandwidth: this kernel runs 16 consumer warps per CTA
+// (two CTAs per SM) and gives each thread NQ = b / 512 queues over positions
+// t + 512 q modulo b (used for b >= 512, one lane per bucket).  A thread sees
+// 16 elements per 8192-element tile, half the chain of the 8-warp layout, and
+// an SM holds twice the warps to overlap the chains.  Stage 2 and the merge
+// run on the first kThreads threads.
+constexpr int kWideConsumers = 512;
+constexpr int kWideWarps = kWideConsumers / 32;
+constexpr int kWideThreads = kWideConsumers + 32;  // consumers + one producer warp
+
+__device__ __forceinline__ void consumer_sync_wide() {
+  asm volatile("bar.sync 2, %0;" ::"r"(kWideConsumers) : "memory");
+}
+
+template <int KB, typename T, int NQ>
+__device__ __forceinline__ void select_tile_wide(Queues<KB, NQ>& q, const T* tile, uint32_t c,
+                                                 uint32_t pos_tile) {
+  constexpr int CT = kWideConsumers;
+  constexpr int U = kTile / CT;  // 16 elements per thread
+  const int t = threadIdx.x;
+  float x[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const bool valid = static_cast<uint32_t>(t + CT * u) < c;
+    x[u] = valid ? to_f32(tile[t + CT * u]) : __int_as_float(0x7f800000);
+  }
+  const uint32_t base = pos_tile + static_cast<uint32_t>(t);
+  if (!(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
+    // NaN or -inf somewhere in this thread's elements: exact update, in order.
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (static_cast<uint32_t>(t + CT * u) >= c) continue;
+      const uint32_t pos = base + static_cast<uint32_t>(CT * u);
+      if (u % NQ == 0)
+        q.template insert_exact<0>(x[u], pos);
+      else
+        q.template insert_exact<(NQ > 1 ? 1 : 0)>(x[u], pos - 1u);
+    }
+    return;
+  }
+  uint32_t mask[NQ];
+  float thr[NQ];
+#pragma unroll
+  for (int v = 0; v < NQ; ++v) {
+    mask[v] = 0u;
+    thr[v] = q.val[v][KB - 1];
+  }
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+    mask[u % NQ] |=
+        (static_cast<uint32_t>(t + CT * u) < c && x[u] > thr[u % NQ]) ? (1u << u) : 0u;
+  // Survivors, software-pipelined as in select_tile_sparse.
+  const T* tt = tile + t;
+#pragma unroll
+  for (int v = 0; v < NQ; ++v) {
+    if (mask[v]) {
+      int u = __ffs(mask[v]) - 1;
+      mask[v] &= mask[v] - 1u;
+      float xc = to_f32(tt[CT * u]);
+      for (;;) {
+        const bool more = mask[v] != 0u;
+        const int un = more ? __ffs(mask[v]) - 1 : u;
+        const float xn = to_f32(tt[CT * un]);
+        if (v == 0)
+          q.template insert_fast<0>(xc, base + static_cast<uint32_t>(CT * u));
+        else
+          q.template insert_fast<(NQ > 1 ? 1 : 0)>(xc, base + static_cast<uint32_t>(CT * u) - 1u);
+        if (!more) break;
+        mask[v] &= mask[v] - 1u;
+        u = un;
+        xc = xn;
+      }
+    }
+  }
+}
+
+template <typename T, int KB, int NQ, bool SAMPLE = false>
+__global__ void __launch_bounds__(kWideThreads, 2) bucket_select_wide(SelectArgs<T> p, int stages,
+                                                                   int cand_cap) {
+  constexpr int kTileElems = Elem<T>::kPerTile;
+  constexpr int NL = kWideConsumers * NQ;  // register queues (lanes) per CTA
+  extern __shared__ __align__(128) unsigned char smem[];
+  const SelectSmem L{stages, KB, cand_cap, NL};
+  T* ring = reinterpret_cast<T*>(smem);
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes() + L.cand_bytes());
+  uint64_t* empty = full + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  int* piece_flag = reinterpret_cast<int*>(empty + stages) + 1;
+
+  const RowSplit& rs = p.rs;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t s0 = cta_start(rs, blockIdx.x);
+  const int64_t e0 = cta_start(rs, blockIdx.x + 1);
+  const int64_t n = rs.n;
+
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, kWideWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait_then_release();
+
+  auto tile_len = [&](int64_t g) -> int64_t {
+    const int64_t rowend = (g / n + 1) * n;
+    int64_t c = e0 - g;
+    if (rowend - g < c) c = rowend - g;
+    return c < kTileElems ? c : kTileElems;
+  };
+
+  if (warp == kWideWarps) {  // ---------------- producer
+    if (lane == 0) {
+      int64_t g = s0, t = 0;
+      int st = 0;
+      uint32_t ph = 0;
+      while (g < e0) {
+        const int64_t c = tile_len(g);
+        if (t >= stages && !mbar_wait_or_abort(empty + st, ph ^ 1u, abort_flag)) break;
+        const uint32_t bytes = static_cast<uint32_t>(c * static_cast<int64_t>(sizeof(T)));
+        mbar_expect_tx(full + st, bytes);
+        bulk_g2s(ring + static_cast<size_t>(st) * kTileElems, p.x + g, bytes, full + st);
+        g += c;
+        ++t;
+        if (++st == stages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      if (*abort_flag) {
+        for (int64_t u = (t > stages ? t - stages : 0); u < t; ++u)
+          mbar_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), 100000000ull);
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers
+  Queues<KB, NQ> q;
+  int st = 0;
+  uint32_t ph = 0;
+  int64_t g = s0;
+  while (g < e0) {
+    const int64_t r = g / n;
+    const int64_t row0 = r * n;
+    const int64_t a = g - row0;
+    const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
+    const uint32_t len = static_cast<uint32_t>(pend - g);
+    q.reset();
+    for (uint32_t done = 0; done < len;) {
+      const uint32_t c =
+          (len - done) < static_cast<uint32_t>(kTileElems) ? (len - done) : kTileElems;
+      const bool ok = __any_sync(0xffffffffu,
+                                 !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
+      if (ok) {
+        const T* stage_tile = ring + static_cast<size_t>(st) * kTileElems;
+#pragma unroll
+        for (int h = 0; h < kTileElems / kTile; ++h) {
+          const uint32_t hoff = static_cast<uint32_t>(h * kTile);
+          if (hoff < c)
+            select_tile_wide<KB, T, NQ>(q, stage_tile + hoff, c - hoff,
+                                        static_cast<uint32_t>(a) + done + hoff);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + st);
+      if (++st == stages) {
+        st = 0;
+        ph ^= 1u;
+      }
+      done += c;
+    }
+    g = pend;
+#pragma unroll
+    for (int v = 0; v < NQ; ++v)
+      q.store(v, lanebuf + static_cast<size_t>(tid + kWideConsumers * v) * KB);
+    consumer_sync_wide();
+    if (tid < kThreads)
+      finish_piece<KB, kGatherInput, T>(rs, p.b, p.k, r, a, static_cast<int64_t>(len), lanebuf,
+                                        cand, p.x + row0, p.out_vals, p.out_idx, piece_flag, NL,
+                                        SAMPLE ? p.tail : SampleTail{nullptr, nullptr, 1.0f});
+    consumer_sync_wide();
+  }
+}
+
 template <typename T, int KB>
 __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs<T> p, int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];

@@ -20,7 +20,7 @@
 namespace tk {
 
 // ------------------------------------------------------------------ queues
-// Four register queues per thread.  Queue v keeps the best KB elements offered
+// Register queues per thread.  Queue v keeps the best KB elements offered
 // to it, best-first, as (value, index) in the float domain; an empty slot holds
 // -inf with index kEmpty.  Elements reach a queue in increasing index order, so
 // "x ranks above slot s" needs no index comparison: with x neither NaN nor -inf
@@ -32,16 +32,20 @@ namespace tk {
 // Stored indices are "base" positions: queue v of a thread stores p - v for an
 // element at position p, so one base per float4 serves its four queues; the
 // true position is restored in store().
-template <int KB>
+//
+// NQ queues per thread: four for the float4 layout (k_b <= 2), one or two for
+// the wide k_b > 2 kernel.  The four-queue members (offer4, offer_tile, ...)
+// exist only for NQ == 4.
+template <int KB, int NQ = 4>
 struct Queues {
-  float val[4][KB];
-  uint32_t idx[4][KB];
+  float val[NQ][KB];
+  uint32_t idx[NQ][KB];
 
   static constexpr uint32_t kEmpty = 0xffffffffu;
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < NQ; ++v) {
 #pragma unroll
       for (int s = 0; s < KB; ++s) {
         val[v][s] = __int_as_float(0xff800000);
@@ -151,7 +155,7 @@ struct Queues {
     for (int s = 0; s < KB; ++s) {
       uint64_t p = 0;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < NQ; ++w) {
         if (w == v && idx[w][s] != kEmpty)
           p = pack(order_key(val[w][s]), idx[w][s] + static_cast<uint32_t>(w));
       }

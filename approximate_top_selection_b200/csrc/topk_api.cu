@@ -97,6 +97,7 @@ struct Plan {
   int64_t units = 0;
   size_t ws_tickets = 0;  // bytes
   size_t ws_slots = 0;    // bytes
+  int wide_nq = 0;        // k_b > 2 fast path: queues per thread of the 16-warp kernel
   size_t workspace() const { return ws_tickets + ws_slots; }
 };
 
@@ -195,20 +196,40 @@ int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, 
   return static_cast<int>(G);
 }
 
+#ifndef TOPK_WIDE_SPARSE
+#define TOPK_WIDE_SPARSE 1
+#endif
+
 template <typename T, int KB>
 int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
   const int C = b * KB;
   pl->cand_cap = sort_capacity(C);
   pl->align = fast ? Elem<T>::kAlign : 1;
-  pl->stages = fast ? fit_stages(SelectSmem{0, KB, pl->cand_cap, select_lanes(KB, b)}, 2) : 0;
+  pl->wide_nq = 0;
   int per_sm = 0;
-  if (fast) {
+  if (fast && KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers) {
+    // k_b > 2 with b >= 512: the 16-warp kernel, one lane per bucket (b lanes).
+    // Smaller b keeps the 8-warp kernel, whose 256 lanes split a bucket over
+    // fewer queues (fewer inserts).
+    pl->wide_nq = b > kWideConsumers ? b / kWideConsumers : 1;
+    const int nl = kWideConsumers * pl->wide_nq;
+    pl->stages = fit_stages(SelectSmem{0, KB, pl->cand_cap, nl}, 2);
+    SelectSmem L{pl->stages, KB, pl->cand_cap, nl};
+    pl->smem = L.total();
+    if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+    int rc = pl->wide_nq == 1
+                 ? occupancy(bucket_select_wide<T, (KB > 2 ? KB : 3), 1>, kWideThreads, pl->smem, &per_sm)
+                 : occupancy(bucket_select_wide<T, (KB > 2 ? KB : 3), 2>, kWideThreads, pl->smem, &per_sm);
+    if (rc) return rc;
+  } else if (fast) {
+    pl->stages = fit_stages(SelectSmem{0, KB, pl->cand_cap, select_lanes(KB, b)}, 2);
     SelectSmem L{pl->stages, KB, pl->cand_cap, select_lanes(KB, b)};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
     int rc = occupancy(bucket_select_tma<T, KB>, kPipeThreads, pl->smem, &per_sm);
     if (rc) return rc;
   } else {
+    pl->stages = 0;
     SelectSmem L{0, KB, pl->cand_cap, kLanes};
     pl->smem = L.total();
     if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
@@ -344,6 +365,23 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 
 template <typename T, int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
+  if constexpr (KB > 2) {
+    if (fast && pl.wide_nq > 0) {
+      const bool sample = a.tail.token != nullptr;
+      auto go = [&](auto kernel) -> int {
+        int rc = prepare_kernel(kernel);
+        if (rc) return rc;
+        return launch_pdl(kernel, dim3(pl.G), dim3(kWideThreads), pl.smem, st, a, pl.stages,
+                          pl.cand_cap);
+      };
+      if constexpr (std::is_same<T, float>::value) {
+        if (sample)
+          return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1, true>)
+                                 : go(bucket_select_wide<T, KB, 2, true>);
+      }
+      return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1>) : go(bucket_select_wide<T, KB, 2>);
+    }
+  }
   if constexpr (std::is_same<T, float>::value) {
     if (fast && a.tail.token != nullptr) {
       int rc = prepare_kernel(bucket_select_tma<T, KB, true>);

@@ -354,3 +354,33 @@ def test_bf16_special_values_and_general_path(oracle_mod):
 def test_bf16_vocab_config(oracle_mod):
     x = inputs.vocab_logits(256, 131072, inputs.SEEDS["vocab"]).to(torch.bfloat16)
     _bf16_check(x, 50, 512, 1, oracle_mod)
+
+
+# ------------------------------------------------------------------ k_b > 2, b >= 512
+@pytest.mark.parametrize("b", [512, 1024])
+@pytest.mark.parametrize("kb", [3, 4])
+def test_wide_kernel_shapes(oracle_mod, b, kb):
+    """The 16-warp k_b > 2 kernel (b >= 512): whole rows, rows split across
+    CTAs, ragged tails, special values, fp32 and bf16 rows, and its sampling
+    variant."""
+    for rows, n, k, kind in [(16, 65536, 512, "u"), (3, 400000, 700, "u"), (40, 8196, 100, "s"),
+                             (300, 20000, 2000, "n"), (2, 4100, 4096, "i")]:
+        seed = 900 + rows + n + b + kb
+        if kind == "u":
+            x = inputs.uniform_rows(rows, n, seed)
+        elif kind == "n":
+            x = inputs.normal_rows(rows, n, seed)
+        elif kind == "i":
+            x = inputs.integer_rows(rows, n, 9, seed)
+        else:
+            x = inputs.special_rows(rows, n, seed)
+        check_bucketed(x, k, b, kb, oracle_mod)
+        if kind != "s":
+            _bf16_check(x.to(torch.bfloat16), k, b, kb, oracle_mod)
+    x = inputs.vocab_logits(8, 65536, 77 + b + kb)
+    u = torch.rand(8, generator=torch.Generator().manual_seed(kb))
+    tok, v, i = atk.topk_sample(x.to(DEV), 64, b, kb, 1.0, u.to(DEV))
+    ov, oi = oracle_mod.bucketed(x.numpy(), 64, b, kb)
+    assert np.array_equal(i.cpu().numpy(), oi)
+    otok, margin = oracle_mod.sample_rows(ov, oi, 1.0, u.numpy().astype(np.float64))
+    assert np.all((tok.cpu().numpy() == otok) | (margin < 1e-5))
