@@ -241,6 +241,8 @@ def _kernel_name(cfg) -> str:
         return "score_select_umma" if _uses_tensor_cores(cfg) else "score_select_gemv"
     if cfg["kind"] == "rerank":
         return "rerank_kernel"
+    if cfg["kb"] > 2 and cfg["b"] >= 512:
+        return "bucket_select_wide"  # the 16-warp k_b > 2 kernel
     return "bucket_select_tma"
 
 
@@ -473,6 +475,7 @@ def run_ours(args, world, rank, local):
 # files are unchanged since the capture.
 _KERNEL_SOURCES = {
     "bucket_select_tma": ("common.cuh", "select_core.cuh", "bucket_select.cuh"),
+    "bucket_select_wide": ("common.cuh", "select_core.cuh", "bucket_select.cuh"),
     "score_select_gemv": ("common.cuh", "select_core.cuh", "score_gemv.cuh"),
     "score_select_umma": ("common.cuh", "select_core.cuh", "score_umma.cuh"),
     "rerank_kernel": ("common.cuh", "select_core.cuh", "rerank.cuh"),
