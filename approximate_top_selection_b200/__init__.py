@@ -11,4 +11,4 @@ CUDA library libtopk_b200.so (build: `python -m approximate_top_selection_b200.b
 from ._binding import (  # noqa: F401
     TOPK_EINVAL, TOPK_ECUDA, TOPK_ESCRATCH, TOPK_EUNSUPPORTED, TOPK_EWORKSPACE, TOPK_OK, TOPK_OP_BUCKETED,
     TOPK_OP_BUCKETED_BF16, TOPK_OP_EXACT, TOPK_OP_SCORE, TopkError, library_path, load_library, score_rerank, score_topk,
-    topk_bucketed, topk_bucketed_bf16, topk_bucketed_merge, topk_bucketed_noalloc, topk_sample, topk_sample_rows, topk_device_status, topk_exact, topk_status_string, topk_workspace_bytes)
+    topk_bucketed, topk_bucketed_bf16, topk_bucketed_merge, topk_bucketed_noalloc, topk_sample, topk_sample_rows, topk_device_status, topk_exact, topk_selftest_wait_timeout, topk_status_string, topk_workspace_bytes)

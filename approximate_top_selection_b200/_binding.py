@@ -63,6 +63,8 @@ def load_library():
             lib.topk_bucketed_merge.restype = i32
             lib.score_rerank.argtypes = [p, i64, i32, p, i64, i64, p, i32, i32, p, p, p, p]
             lib.score_rerank.restype = i32
+            lib.topk_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
+            lib.topk_selftest_wait_timeout.restype = i32
             f32 = ctypes.c_float
             lib.topk_sample_rows.argtypes = [p, p, i64, i32, f32, p, p, p]
             lib.topk_sample_rows.restype = i32
@@ -403,6 +405,15 @@ def score_topk(q: torch.Tensor, K: torch.Tensor, k: int, b: int, kb: int, *,
     if return_scores:
         return out_vals, out_idx, scores
     return out_vals, out_idx
+
+
+def topk_selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Queue a bounded wait that is sure to expire (see the header); the next
+    topk_device_status() then reports the expiry."""
+    lib = load_library()
+    with _OnDevice(torch.device("cuda", torch.cuda.current_device())) as on:
+        _check(lib.topk_selftest_wait_timeout(int(limit_ns), _stream_handle(stream, on.index)),
+               "topk_selftest_wait_timeout")
 
 
 def topk_device_status() -> int:

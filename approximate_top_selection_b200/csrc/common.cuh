@@ -193,4 +193,17 @@ __host__ __device__ __forceinline__ int part_of(int64_t g, int64_t units, int G,
   return static_cast<int>(c);
 }
 
+// Bounded-wait self-test: one thread waits on an mbarrier that nothing will
+// complete, for at most limit_ns, then returns; the expiry is recorded in the
+// device status like any other expired wait.  Exercises the failure path of
+// every bounded wait without a fault, a trap or a hang.
+__global__ void wait_timeout_probe(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait(&bar, 0u, limit_ns);
+  }
+}
+
 }  // namespace tk

@@ -838,6 +838,13 @@ int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_
   }
 }
 
+int topk_selftest_wait_timeout(unsigned long long limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > kWaitLimitNs) return TOPK_EINVAL;
+  clear_launch_error();
+  wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? TOPK_OK : TOPK_ECUDA;
+}
+
 int topk_device_status(int* status_out) {
   if (!status_out) return TOPK_EINVAL;
   if (cudaDeviceSynchronize() != cudaSuccess) return TOPK_ECUDA;

@@ -224,6 +224,15 @@ int score_topk(const uint16_t *q_dev, int64_t rows, int d, const uint16_t *K_dev
 int topk_bucketed_noalloc(const float *scores_dev, int64_t rows, int64_t n, int k, int b, int kb,
                           float *out_vals_dev, int32_t *out_idx_dev, void *stream);
 
+/* Self-test of the bounded waits (no counterpart in the paper): one thread
+ * waits, for at most limit_ns nanoseconds (1e3 .. 2e9, else TOPK_EINVAL), on
+ * a barrier that nothing completes, gives up and records TOPK_DEV_WAIT_TIMEOUT
+ * in the device status, exactly as an expired wait of a selection kernel does.
+ * The GPU neither faults nor hangs and the context stays usable; it lets a
+ * caller check its error handling for expired waits.  Asynchronous on
+ * `stream`. */
+int topk_selftest_wait_timeout(unsigned long long limit_ns, void *stream);
+
 /* Human-readable name of a topk_status value (static string). */
 const char *topk_status_string(int status);
 

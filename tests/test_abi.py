@@ -113,6 +113,13 @@ def test_sampling_rejects_bad_arguments_on_host(lib):
     assert lib.topk_sample(None, 1, 8, 4, 2, 1, 1.0, p, p, p, p, None, 0, None) == E
 
 
+def test_selftest_rejects_bad_limits_on_host(lib):
+    E = atk.TOPK_EINVAL
+    assert lib.topk_selftest_wait_timeout(0, None) == E
+    assert lib.topk_selftest_wait_timeout(999, None) == E
+    assert lib.topk_selftest_wait_timeout(3 * 10 ** 9, None) == E
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
 
