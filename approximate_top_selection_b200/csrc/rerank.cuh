@@ -13,7 +13,9 @@
 //
 // One CTA per row.  Duplicate indices (overlapping supports) are dropped by a
 // shared-memory hash set (first insert wins; duplicates carry identical
-// scores, so which copy survives does not matter).  A group of D/16 lanes
+// scores, so which copy survives does not matter) and the distinct candidates
+// are listed densely, so no gather pass is spent on an empty or repeated slot
+// and Stage 2 sees only real candidates.  A group of D/16 lanes
 // scores one candidate: each lane holds 16 query values in registers and
 // loads 16 key values with two 16-byte loads (two candidates in flight per
 // group; four CTAs per SM so that 512 rows fit one wave), and the group sums with
@@ -61,7 +63,7 @@ __global__ void __launch_bounds__(kThreads, TOPK_RERANK_MIN_CTAS) rerank_kernel(
   const int C = p.c;
   const int cap = sort_capacity(C);
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem);                      // [cap]
-  int32_t* table = reinterpret_cast<int32_t*>(smem + stage2_bytes(C));     // hash set of indices
+  int32_t* table = reinterpret_cast<int32_t*>(smem + stage2_bytes(C));  // hash set, then the list
   const int H = rerank_table_size(C);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait_then_release();
@@ -95,7 +97,33 @@ __global__ void __launch_bounds__(kThreads, TOPK_RERANK_MIN_CTAS) rerank_kernel(
   if (bad) atomicOr(&g_device_status, 2);
   group_sync(kThreads);
 
-  // 2. exact scores of the owned slots
+  // 2. the (slot, index) list of the owned slots replaces the hash set, and
+  //    the marks are cleared so that cand can take the packed words densely
+  int* owned_count = reinterpret_cast<int*>(table + H);
+  if (tid == 0) *owned_count = 0;
+  group_sync(kThreads);
+  int32_t* olist = table;  // [2 m]
+  for (int base = warp * 32; base < C; base += kThreads) {
+    const int j = base + lane;
+    const bool own = j < C && cand[j] != 0ull;
+    const unsigned mk = __ballot_sync(0xffffffffu, own);
+    int at = 0;
+    if (lane == 0 && mk) at = atomicAdd(owned_count, __popc(mk));
+    at = __shfl_sync(0xffffffffu, at, 0) + __popc(mk & ((1u << lane) - 1u));
+    if (own) {
+      olist[2 * at] = j;
+      olist[2 * at + 1] = __ldg(ci + j);
+    }
+    if (j < C) {
+      cand[j] = 0ull;
+      if (!own && p.out_scores)
+        p.out_scores[r * static_cast<int64_t>(C) + j] = __int_as_float(0xff800000);
+    }
+  }
+  group_sync(kThreads);
+  const int m = *owned_count;
+
+  // 3. exact scores of the m distinct candidates
   const int g = lane / G, gl = lane % G;
   const uint16_t* qr = p.q + r * static_cast<int64_t>(D) + gl * 16;
   float qv[16];
@@ -114,22 +142,22 @@ __global__ void __launch_bounds__(kThreads, TOPK_RERANK_MIN_CTAS) rerank_kernel(
   // before any is used, so a warp keeps 2R 16-byte loads per lane outstanding.
   constexpr int R = TOPK_RERANK_INFLIGHT;
   constexpr int STEP = (kThreads / 32) * PER_WARP;  // candidates per CTA pass
-  for (int base = warp * PER_WARP; base < C; base += R * STEP) {
+  for (int base = warp * PER_WARP; base < m; base += R * STEP) {
     uint4 ka[R], kb[R];
     int32_t ii[R];
-    bool own[R];
+    bool live[R];
 #pragma unroll
     for (int u = 0; u < R; ++u) {
-      const int j = base + u * STEP + g;
-      own[u] = j < C && cand[j] != 0ull;
-      ii[u] = own[u] ? __ldg(ci + j) : 0;
+      const int e = base + u * STEP + g;
+      live[u] = e < m;
+      ii[u] = live[u] ? olist[2 * e + 1] : 0;
       const uint16_t* kr = Kr + static_cast<int64_t>(ii[u]) * D + gl * 16;
-      ka[u] = own[u] ? __ldg(reinterpret_cast<const uint4*>(kr)) : make_uint4(0, 0, 0, 0);
-      kb[u] = own[u] ? __ldg(reinterpret_cast<const uint4*>(kr + 8)) : make_uint4(0, 0, 0, 0);
+      ka[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(kr)) : make_uint4(0, 0, 0, 0);
+      kb[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(kr + 8)) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < R; ++u) {
-      const int j = base + u * STEP + g;
+      const int e = base + u * STEP + g;
       const uint32_t w[8] = {ka[u].x, ka[u].y, ka[u].z, ka[u].w, kb[u].x, kb[u].y, kb[u].z, kb[u].w};
       float s = 0.0f;
 #pragma unroll
@@ -139,20 +167,17 @@ __global__ void __launch_bounds__(kThreads, TOPK_RERANK_MIN_CTAS) rerank_kernel(
       }
 #pragma unroll
       for (int o = G / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (gl == 0 && j < C) {
-        if (own[u]) {
-          s = s + 0.0f;  // -0 -> +0: a zero score is +0
-          cand[j] = pack(order_key(s), static_cast<uint32_t>(ii[u]));
-        }
-        if (p.out_scores)
-          p.out_scores[r * static_cast<int64_t>(C) + j] = own[u] ? s : __int_as_float(0xff800000);
+      if (gl == 0 && live[u]) {
+        s = s + 0.0f;  // -0 -> +0: a zero score is +0
+        cand[e] = pack(order_key(s), static_cast<uint32_t>(ii[u]));
+        if (p.out_scores) p.out_scores[r * static_cast<int64_t>(C) + olist[2 * e]] = s;
       }
     }
   }
   group_sync(kThreads);
 
-  // 3. exact top-k of the scored candidates
-  stage2<kFromKey, float>(cand, C, p.k, nullptr, p.out_vals + r * static_cast<int64_t>(p.k),
+  // 4. exact top-k of the m scored candidates
+  stage2<kFromKey, float>(cand, m, p.k, nullptr, p.out_vals + r * static_cast<int64_t>(p.k),
                           p.out_idx + r * static_cast<int64_t>(p.k));
 }
 
