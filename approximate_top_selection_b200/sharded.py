@@ -1,5 +1,8 @@
 """Rows cut into column slices across ranks (vocabulary- or entity-parallel).
 
+split_row_topk takes score rows; split_score_topk takes the key matrices of
+the fused scorers, split by keys.
+
 Each rank holds columns [offset, offset + n_local) of the same rows.  It runs
 the bucketed selection on its slice, the (value, index) candidate lists of all
 ranks are all-gathered -- the one exchange of the method when a row is split
@@ -70,5 +73,21 @@ def split_row_topk(x_local: torch.Tensor, offset: int, n_total: int, k: int, b: 
     """
     v, i = _binding.topk_bucketed(x_local, k, b, kb)
     offsets = gather_offsets(offset, group, device=x_local.device)
+    V, I = gather_candidates(v, i, group)
+    return _binding.topk_bucketed_merge(V, I, n_total, k, b, kb, part_offsets=offsets)
+
+
+def split_score_topk(q: torch.Tensor, K_local: torch.Tensor, offset: int, n_total: int, k: int, b: int,
+                     kb: int, group=None):
+    """Fused scoring and bucketed top-k with the keys split by rows across the
+    ranks (entity- or sequence-parallel): this rank holds keys
+    [offset, offset + n_local) of every row's key matrix.
+
+    q: [rows, d] bf16, the same on every rank; K_local: [rows, n_local, d] or
+    [n_local, d] bf16.  Returns (values, global indices) [rows, k] on every rank,
+    equal to score_topk over the whole key matrices.
+    """
+    v, i = _binding.score_topk(q, K_local, k, b, kb)
+    offsets = gather_offsets(offset, group, device=q.device)
     V, I = gather_candidates(v, i, group)
     return _binding.topk_bucketed_merge(V, I, n_total, k, b, kb, part_offsets=offsets)

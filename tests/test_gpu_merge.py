@@ -155,3 +155,35 @@ def test_merge_skips_and_flags_out_of_range_indices(oracle_mod):
     ov, oi = _oracle_merge(oracle_mod, vals, clean, offs, 20, 8, 2)
     assert np.array_equal(mi.cpu().numpy(), oi)
     assert np.array_equal(bits(mv.cpu()), bits(ov))
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_split_keys_merge_equals_fused_single_pass(oracle_mod, shared):
+    """Entity-parallel emulation on one GPU: the key matrices cut into slices,
+    score_topk on each slice, then the merge.  The result equals the bucketed
+    selection over the slices' own fp32 scores bit for bit (the oracle on those
+    scores); a slice may sum a dot product in another fp32 order than the whole
+    matrix does, so the scores themselves are checked against each other to
+    the scoring tolerance."""
+    rows, n, d, k, b, kb = (64, 65536, 256, 100, 1024, 1) if shared else (8, 20000, 128, 256, 128, 2)
+    q = inputs.bf16_normal((rows, d), 1.0, 0xC0 + n, device=DEV)
+    K = inputs.bf16_normal((n, d) if shared else (rows, n, d), d ** -0.5, 0xC1 + n, device=DEV)
+    cuts = [0, n // 3, n // 3 + 4096 + 5, n] if not shared else [0, 16384, 40960, n]
+    vs, is_, ss = [], [], []
+    for s0, e0 in zip(cuts[:-1], cuts[1:]):
+        Ks = K[s0:e0].contiguous() if shared else K[:, s0:e0].contiguous()
+        v, i, sc = atk.score_topk(q, Ks, k, b, kb, return_scores=True)
+        vs.append(v)
+        is_.append(i)
+        ss.append(sc)
+    mv, mi = atk.topk_bucketed_merge(torch.stack(vs), torch.stack(is_), n, k, b, kb,
+                                     part_offsets=cuts[:-1])
+    torch.cuda.synchronize()
+    slice_scores = torch.cat(ss, dim=1).cpu().numpy()
+    ov, oi = oracle_mod.bucketed(slice_scores, k, b, kb)
+    assert np.array_equal(mi.cpu().numpy(), oi)
+    assert np.array_equal(bits(mv.cpu()), bits(ov))
+    _, _, fs = atk.score_topk(q, K, k, b, kb, return_scores=True)
+    full = fs.cpu().numpy().astype(np.float64)
+    # fp32 sums of the same products in another order: a few ulps of sum(abs(terms))
+    assert np.all(np.abs(slice_scores - full) <= 1e-5 + 1e-5 * np.abs(full))
