@@ -293,6 +293,40 @@ __device__ __forceinline__ void block_sort_desc(uint64_t (&v)[EPT], uint64_t* xc
   bitonic_sizes<EPT, 2>(v, xchg);
 }
 
+// Bitonic network on the 32 * EPT keys of one warp, strided (lane l holds
+// elements j * 32 + l): strides below 32 are shuffles, larger ones register
+// swaps; no shared memory, no block barrier.
+template <int EPT, int SIZE, int STRIDE>
+__device__ __forceinline__ void warp_bitonic_round(uint64_t (&v)[EPT], int lane) {
+  if constexpr (STRIDE >= 32) {
+    constexpr int DJ = STRIDE / 32;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      if ((j & DJ) == 0) {
+        const bool desc = ((j * 32) & SIZE) == 0;
+        const uint64_t a = v[j], b = v[j | DJ];
+        v[j] = desc ? umax64(a, b) : umin64(a, b);
+        v[j | DJ] = desc ? umin64(a, b) : umax64(a, b);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * 32 + lane;
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, v[j], STRIDE);
+      const bool keep_max = ((e & SIZE) == 0) == ((lane & STRIDE) == 0);
+      v[j] = keep_max ? umax64(v[j], o) : umin64(v[j], o);
+    }
+  }
+  if constexpr (STRIDE > 1) warp_bitonic_round<EPT, SIZE, STRIDE / 2>(v, lane);
+}
+
+template <int EPT, int SIZE>
+__device__ __forceinline__ void warp_bitonic_sizes(uint64_t (&v)[EPT], int lane) {
+  warp_bitonic_round<EPT, SIZE, SIZE / 2>(v, lane);
+  if constexpr (SIZE < 32 * EPT) warp_bitonic_sizes<EPT, SIZE * 2>(v, lane);
+}
+
 // Value of an output candidate: from its key, except that a zero or NaN is
 // re-read from the input row so that -0.0 and NaN payloads keep their bits.
 // V is the element type of the output: float, or uint16_t holding bf16 bits
@@ -367,6 +401,61 @@ __host__ __device__ __forceinline__ size_t stage2_bytes(int C) {
 template <ValueSource VS, typename V>
 __device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const V* xrow, V* ov,
                                                   int32_t* oi);
+
+// Stage 2 for a small k (k <= M = 32 * EPT, C <= 8 M): every warp sorts its M
+// candidates in registers, then in three rounds warp w < h takes the list of
+// warp w + h from shared memory and keeps the M best of the two (the bitonic
+// merge: max(own[e], partner[M-1-e]) is a bitonic sequence holding the M
+// best, and log2(M) more rounds sort it).  Warp 0 ends with the M best,
+// sorted, and writes the first k.  Fewer exchanges and barriers than sorting
+// all C when only k of them are wanted.
+template <int EPT, int VS, typename V>
+__device__ __noinline__ void finalize_row_topk_warps(uint64_t* cand, int C, int k, const V* xrow,
+                                                     V* ov, int32_t* oi) {
+  constexpr int M = 32 * EPT;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  uint64_t v[EPT];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = w * M + j * 32 + lane;
+    v[j] = e < C ? cand[e] : 0ull;
+  }
+  warp_bitonic_sizes<EPT, 2>(v, lane);
+  group_sync(kThreads);  // every candidate has been read
+#pragma unroll
+  for (int h = kThreads / 64; h >= 1; h >>= 1) {
+    if (w >= h && w < 2 * h) {
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) cand[(w - h) * M + j * 32 + lane] = v[j];
+    }
+    group_sync(kThreads);
+    if (w < h) {
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int e = j * 32 + lane;
+        v[j] = umax64(v[j], cand[w * M + (M - 1 - e)]);
+      }
+      warp_bitonic_round<EPT, 2 * M, M / 2>(v, lane);  // descending merge of a bitonic sequence
+    }
+    group_sync(kThreads);
+  }
+  if (w == 0) {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * 32 + lane;
+      if (e < k) {
+        if (v[j]) {
+          ov[e] = candidate_value<VS, V>(v[j], xrow);
+          oi[e] = static_cast<int32_t>(packed_idx(v[j]));
+        } else {
+          ov[e] = negative_infinity<V>();
+          oi[e] = -1;
+        }
+      }
+    }
+  }
+  group_sync(kThreads);
+}
 
 // Stage 2 when the candidates far outnumber k: find the k-th largest packed
 // key with 8-bit radix histograms (most significant digit first; keys are
@@ -560,9 +649,23 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
 
 // Stage 2 entry of the streaming kernels: select first when that shrinks the
 // sort (at least 1024 candidates and k under half of them), else sort all.
+#ifndef TOPK_WARP_TOPK
+#define TOPK_WARP_TOPK 1
+#endif
 template <ValueSource VS, typename V>
 __device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xrow, V* ov,
                                        int32_t* oi) {
+  if (TOPK_WARP_TOPK && C > k && C <= 8 * kThreads) {
+    const int ept = sort_capacity(C) / kThreads;
+    if (k <= 32 * ept) {
+      switch (ept) {
+        case 2: finalize_row_topk_warps<2, VS, V>(cand, C, k, xrow, ov, oi); return;
+        case 4: finalize_row_topk_warps<4, VS, V>(cand, C, k, xrow, ov, oi); return;
+        case 8: finalize_row_topk_warps<8, VS, V>(cand, C, k, xrow, ov, oi); return;
+        default: break;
+      }
+    }
+  }
   if (C >= 1024 && 2 * k <= C && C <= 16 * kThreads) {
     switch (sort_capacity(C) / kThreads) {
       case 4: finalize_row_select<4, VS, V>(cand, C, k, xrow, ov, oi); return;
