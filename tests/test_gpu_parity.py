@@ -384,3 +384,15 @@ def test_wide_kernel_shapes(oracle_mod, b, kb):
     assert np.array_equal(i.cpu().numpy(), oi)
     otok, margin = oracle_mod.sample_rows(ov, oi, 1.0, u.numpy().astype(np.float64))
     assert np.all((tok.cpu().numpy() == otok) | (margin < 1e-5))
+
+
+@pytest.mark.parametrize("b,kb,k", [(1024, 4, 3000), (1024, 4, 16384), (1024, 3, 2500), (1000, 4, 3500)])
+def test_largest_candidate_sets_and_k(oracle_mod, b, kb, k):
+    """The support limits: b = 1024 buckets of k_b = 4 (4096 candidates: the
+    shared-memory sort of Stage 2), k up to 16384 (padding past the 4096
+    candidates), b = 1000 (general kernel), one long row and rows split over
+    CTAs, fp32 and bf16."""
+    for rows, n in [(2, 1000000), (24, 65536)]:
+        x = inputs.uniform_rows(rows, n, 4242 + b + kb + k + n)
+        check_bucketed(x, k, b, kb, oracle_mod)
+        _bf16_check(x.to(torch.bfloat16), k, b, kb, oracle_mod)

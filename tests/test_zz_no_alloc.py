@@ -31,6 +31,7 @@ SHAPES = [
     (3, 400000, 100, 512, 2, "normal"),     # long rows split across CTAs (fast path)
     (2500, 1001, 20, 50, 2, "uniform"),     # many rows per CTA, cut rows (general path)
     (2, 1 << 20, 300, 256, 4, "ties"),      # heavy ties, split rows
+    (3, 600000, 512, 512, 4, "uniform"),    # the 16-warp k_b > 2 kernel, split rows
 ]
 
 
