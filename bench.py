@@ -247,8 +247,9 @@ def _kernel_name(cfg) -> str:
 
 
 def _launches_per_step(cfg) -> int:
-    # the tensor-core path adds a Stage-2 kernel, sampling adds the draw
-    return 2 if _uses_tensor_cores(cfg) or cfg.get("sample") else 1
+    # the tensor-core path adds a Stage-2 kernel; the sampling draw runs inside
+    # the selection kernel
+    return 2 if _uses_tensor_cores(cfg) else 1
 
 
 def _rotations(w: Workload) -> int:

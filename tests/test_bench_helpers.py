@@ -1,0 +1,64 @@
+"""Host logic of the benchmark contract, on the CPU: which kernel a workload's
+roofline names, the committed DRAM traffic lookup (valid only while the
+kernel's device sources hash to the captured value), input rotation against
+L2, and the launch count claimed per step."""
+import math
+
+import bench
+
+
+def test_every_config_names_a_kernel_with_sources():
+    for name, cfg in bench.CONFIGS.items():
+        k = bench._kernel_name(cfg)
+        assert k in bench._KERNEL_SOURCES, (name, k)
+        assert len(bench._source_hash(k)) == 16
+
+
+def test_kernel_choice_follows_the_library_dispatch():
+    assert bench._kernel_name(bench.CONFIGS["decode"]) == "score_select_gemv"
+    assert bench._kernel_name(bench.CONFIGS["link"]) == "score_select_umma"
+    assert bench._kernel_name(bench.CONFIGS["vocab"]) == "bucket_select_tma"
+    assert bench._kernel_name(bench.CONFIGS["long-b512-kb4"]) == "bucket_select_wide"
+    assert bench._kernel_name(bench.CONFIGS["long-b256-kb4"]) == "bucket_select_tma"
+    assert bench._kernel_name(bench.CONFIGS["decode-rerank"]) == "rerank_kernel"
+
+
+def test_traffic_rows_match_the_current_sources():
+    """Every traffic row of the committed summary refers to a known kernel;
+    a row whose hash is current yields its byte count, others yield None."""
+    rows = 0
+    for line in open(bench.os.path.join(bench.ROOT, "profiles", "traffic.md")):
+        cells = [c.strip() for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 4 and cells[1] in bench._KERNEL_SOURCES:
+            rows += 1
+            got = bench._traffic(cells[0])
+            if cells[2] == bench._source_hash(cells[1]):
+                assert got == int(cells[3])
+            else:
+                assert got is None
+    assert rows >= 4
+    assert bench._traffic("no-such-workload") is None
+
+
+def test_launches_per_step():
+    assert bench._launches_per_step(bench.CONFIGS["link"]) == 2
+    assert bench._launches_per_step(bench.CONFIGS["decode"]) == 1
+    assert bench._launches_per_step(bench.CONFIGS["vocab-sample"]) == 1  # draw fused
+    assert bench._launches_per_step(bench.CONFIGS["vocab"]) == 1
+
+
+class _W:
+    def __init__(self, in_bytes):
+        self.in_bytes = in_bytes
+        self.larger_than_l2 = in_bytes > 126 * 2 ** 20
+
+
+def test_rotations_defeat_l2():
+    assert bench._rotations(_W(4 << 30)) == 1
+    for b in (1 << 17, 64 << 20, 120 << 20):
+        n = bench._rotations(_W(b))
+        assert n >= 2 and n * b >= 3 * 126 * 2 ** 20
+
+
+def test_job_throughput_is_weak_scaling():
+    assert math.isclose(bench.job_throughput(1e9, 2.0, 4), 4 * 1e9 / 2e-3 / 1e9)
