@@ -63,6 +63,10 @@ MUTANTS = [
      "        if (idx[i] < 0)\n            continue;\n        const double w",
      "        const double w",
      [P.pin_sampling_special]),
+    ("pair selection buckets by list position instead of index",
+     "            if (all[t].i % b == j)",
+     "            if (t % b == j)",
+     [P.pin_split_merge]),
     ("re-ranking keeps repeated candidates",
      "                if (seen)\n                    continue;\n",
      "",
