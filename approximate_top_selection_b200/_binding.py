@@ -70,6 +70,8 @@ def load_library():
             lib.topk_sample_rows.restype = i32
             lib.topk_sample.argtypes = [p, i64, i64, i32, i32, i32, f32, p, p, p, p, p, sz, p]
             lib.topk_sample.restype = i32
+            lib.topk_sample_bf16.argtypes = [p, i64, i64, i32, i32, i32, f32, p, p, p, p, p, sz, p]
+            lib.topk_sample_bf16.restype = i32
             lib.topk_status_string.argtypes = [i32]
             lib.topk_status_string.restype = ctypes.c_char_p
             lib.topk_device_status.argtypes = [ctypes.POINTER(ctypes.c_int)]
@@ -342,23 +344,28 @@ def topk_sample_rows(vals: torch.Tensor, idx: torch.Tensor, temperature: float, 
 
 def topk_sample(logits: torch.Tensor, k: int, b: int, kb: int, temperature: float, u: torch.Tensor, *,
                 out_vals=None, out_idx=None, out_token=None, stream=None):
-    """Bucketed top-k of float32 logits [rows, n], then one sampled token per
-    row.  Returns (tokens [rows], values [rows, k], indices [rows, k])."""
+    """Bucketed top-k of float32 or bfloat16 logits [rows, n], then one
+    sampled token per row.  Returns (tokens [rows], values [rows, k] of the
+    logits' dtype, indices [rows, k])."""
     lib = load_library()
-    _cuda(logits, "logits", torch.float32)
+    bf16 = isinstance(logits, torch.Tensor) and logits.dtype == torch.bfloat16
+    _cuda(logits, "logits", torch.bfloat16 if bf16 else torch.float32)
     _cuda(u, "u", torch.float32)
     if logits.dim() != 2 or u.numel() != logits.shape[0]:
         raise ValueError("logits must be [rows, n] and u [rows]")
     rows, n = logits.shape
     with _OnDevice(logits.device) as on:
         sh = _stream_handle(stream, on.index)
-        out_vals, out_idx = _outputs(rows, k, logits.device, out_vals, out_idx)
+        out_vals, out_idx = _outputs(rows, k, logits.device, out_vals, out_idx,
+                                     dtype=torch.bfloat16 if bf16 else torch.float32)
         if out_token is None:
             out_token = torch.empty(rows, dtype=torch.int32, device=logits.device)
         _cuda(out_token, "out_token", torch.int32)
-        nbytes = topk_workspace_bytes(TOPK_OP_BUCKETED, rows, n, k, b, kb)
+        nbytes = topk_workspace_bytes(TOPK_OP_BUCKETED_BF16 if bf16 else TOPK_OP_BUCKETED,
+                                      rows, n, k, b, kb)
         ws = _workspace(nbytes, logits.device, sh)
-        st = lib.topk_sample(logits.data_ptr(), rows, n, k, b, kb, float(temperature), u.data_ptr(),
+        fn = lib.topk_sample_bf16 if bf16 else lib.topk_sample
+        st = fn(logits.data_ptr(), rows, n, k, b, kb, float(temperature), u.data_ptr(),
                              out_token.data_ptr(), out_vals.data_ptr(), out_idx.data_ptr(),
                              ws.data_ptr() if ws is not None else None,
                              ws.numel() if ws is not None else 0, sh)

@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(32 * kSampleWarps)
   pdl_wait_then_release();
   const int64_t r = static_cast<int64_t>(blockIdx.x) * kSampleWarps + (threadIdx.x >> 5);
   if (r >= rows) return;
-  sample_row_warp(vals + r * k, idx + r * k, k, inv_t, __ldg(u + r), token + r);
+  sample_row_warp<float>(vals + r * k, idx + r * k, k, inv_t, __ldg(u + r), token + r);
 }
 
 }  // namespace tk

@@ -684,12 +684,19 @@ __device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xr
 // of positive weight.  Padding (-1) and -inf weigh 0; a NaN or +inf best
 // entry is drawn outright; no candidate draws -1.  Each lane sums a contiguous
 // slice in fp32 and a shuffle scan gives it the weight before its slice.
-// v and ix are plain loads: they may have been written by this CTA.
-__device__ __forceinline__ void sample_row_warp(const float* v, const int32_t* ix, int k,
-                                                float inv_t, float u, int32_t* token) {
+// v and ix are plain loads: they may have been written by this CTA.  V is
+// float, or uint16_t holding bf16 bits (widened to fp32 exactly).
+__device__ __forceinline__ float sample_value(const float* v, int i) { return v[i]; }
+__device__ __forceinline__ float sample_value(const uint16_t* v, int i) {
+  return __uint_as_float(static_cast<uint32_t>(v[i]) << 16);
+}
+
+template <typename V>
+__device__ __forceinline__ void sample_row_warp(const V* v, const int32_t* ix, int k, float inv_t,
+                                                float u, int32_t* token) {
   const int lane = threadIdx.x & 31;
   const int32_t i0 = ix[0];
-  const float v0 = v[0];
+  const float v0 = sample_value(v, 0);
   if (i0 < 0 || v0 != v0 || v0 == __int_as_float(0x7f800000)) {
     if (lane == 0) *token = i0;  // -1 (no candidate), or the NaN / +inf entry
     return;
@@ -698,7 +705,7 @@ __device__ __forceinline__ void sample_row_warp(const float* v, const int32_t* i
   const int beg = min(lane * per, k), end = min(beg + per, k);
   float part = 0.0f;
   for (int i = beg; i < end; ++i)
-    if (ix[i] >= 0) part += expf((v[i] - v0) * inv_t);
+    if (ix[i] >= 0) part += expf((sample_value(v, i) - v0) * inv_t);
   float incl = part;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -711,7 +718,7 @@ __device__ __forceinline__ void sample_row_warp(const float* v, const int32_t* i
   int32_t pick = -1, last = -1;
   for (int i = beg; i < end; ++i) {
     if (ix[i] < 0) continue;
-    const float w = expf((v[i] - v0) * inv_t);
+    const float w = expf((sample_value(v, i) - v0) * inv_t);
     if (w > 0.0f) last = ix[i];
     run += w;
     if (run > target) {
@@ -735,20 +742,19 @@ struct SampleTail {
 
 // Out of line so that the streaming loop of the selection kernels keeps its
 // registers: the draw runs once per row, after Stage 2.
-__device__ __noinline__ void sample_row_warp_call(const float* v, const int32_t* ix, int k,
+template <typename V>
+__device__ __noinline__ void sample_row_warp_call(const V* v, const int32_t* ix, int k,
                                                   float inv_t, float u, int32_t* token) {
-  sample_row_warp(v, ix, k, inv_t, u, token);
+  sample_row_warp<V>(v, ix, k, inv_t, u, token);
 }
 
 // After Stage 2 of row r wrote ov / oi (and the CTA met at a barrier): warp 0
-// draws the row's token.  Float rows only.
+// draws the row's token.
 template <typename V>
 __device__ __forceinline__ void run_sample_tail(const SampleTail& tail, int64_t r, int k,
                                                 const V* ov, const int32_t* oi) {
-  if constexpr (sizeof(V) == 4) {
-    if (tail.token != nullptr && threadIdx.x < 32)
-      sample_row_warp_call(ov, oi, k, tail.inv_t, __ldg(tail.u + r), tail.token + r);
-  }
+  if (tail.token != nullptr && threadIdx.x < 32)
+    sample_row_warp_call<V>(ov, oi, k, tail.inv_t, __ldg(tail.u + r), tail.token + r);
 }
 
 // ------------------------------------------------------------------ pieces

@@ -374,21 +374,17 @@ int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStre
         return launch_pdl(kernel, dim3(pl.G), dim3(kWideThreads), pl.smem, st, a, pl.stages,
                           pl.cand_cap);
       };
-      if constexpr (std::is_same<T, float>::value) {
-        if (sample)
-          return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1, true>)
-                                 : go(bucket_select_wide<T, KB, 2, true>);
-      }
+      if (sample)
+        return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1, true>)
+                               : go(bucket_select_wide<T, KB, 2, true>);
       return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1>) : go(bucket_select_wide<T, KB, 2>);
     }
   }
-  if constexpr (std::is_same<T, float>::value) {
-    if (fast && a.tail.token != nullptr) {
-      int rc = prepare_kernel(bucket_select_tma<T, KB, true>);
-      if (rc) return rc;
-      return launch_pdl(bucket_select_tma<T, KB, true>, dim3(pl.G), dim3(kPipeThreads), pl.smem,
-                        st, a, pl.stages, pl.cand_cap);
-    }
+  if (fast && a.tail.token != nullptr) {
+    int rc = prepare_kernel(bucket_select_tma<T, KB, true>);
+    if (rc) return rc;
+    return launch_pdl(bucket_select_tma<T, KB, true>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st,
+                      a, pl.stages, pl.cand_cap);
   }
   if (fast)
     return launch_pdl(bucket_select_tma<T, KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
@@ -787,6 +783,17 @@ int topk_sample(const float* logits, int64_t rows, int64_t n, int k, int b, int 
   // The draw runs inside the selection kernel, right after each row's Stage 2.
   return run_bucketed<float>(logits, rows, n, k, b, kb, out_vals, out_idx, workspace,
                              workspace_bytes, stream, SampleTail{u, token, 1.0f / temperature});
+}
+
+int topk_sample_bf16(const uint16_t* logits, int64_t rows, int64_t n, int k, int b, int kb,
+                     float temperature, const float* u, int32_t* token, uint16_t* out_vals,
+                     int32_t* out_idx, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!u || !token) return TOPK_EINVAL;
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isfinite(1.0f / temperature))
+    return TOPK_EINVAL;
+  if (k > kMaxK) return TOPK_EUNSUPPORTED;
+  return run_bucketed<uint16_t>(logits, rows, n, k, b, kb, out_vals, out_idx, workspace,
+                                workspace_bytes, stream, SampleTail{u, token, 1.0f / temperature});
 }
 
 int score_topk(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int64_t n,

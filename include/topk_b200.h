@@ -173,6 +173,14 @@ int topk_sample(const float *logits_dev, int64_t rows, int64_t n, int k, int b, 
                 float temperature, const float *u_dev, int32_t *token_dev, float *out_vals_dev,
                 int32_t *out_idx_dev, void *workspace_dev, size_t workspace_bytes, void *stream);
 
+/* topk_sample on bfloat16 logits (raw 16-bit patterns): the selection of
+ * topk_bucketed_bf16 with the same fused draw; a bf16 logit widens to fp32
+ * exactly before the softmax.  out_vals_dev receives bf16 bits. */
+int topk_sample_bf16(const uint16_t *logits_dev, int64_t rows, int64_t n, int k, int b, int kb,
+                     float temperature, const float *u_dev, int32_t *token_dev,
+                     uint16_t *out_vals_dev, int32_t *out_idx_dev, void *workspace_dev,
+                     size_t workspace_bytes, void *stream);
+
 /* Fused selector: score[r][i] = sum_t q[r][t] * K_r[i][t] (bf16 inputs, fp32
  * accumulation; no 1/sqrt(d) scaling), then topk_bucketed on each row of
  * scores -- the sparse-attention selector that scores the current query

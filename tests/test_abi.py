@@ -111,6 +111,9 @@ def test_sampling_rejects_bad_arguments_on_host(lib):
         assert lib.topk_sample(p, 1, 8, 4, 2, 1, t, p, p, p, p, None, 0, None) == E, t
     assert lib.topk_sample(p, 1, 8, 4, 2, 1, 1.0, None, p, p, p, None, 0, None) == E
     assert lib.topk_sample(None, 1, 8, 4, 2, 1, 1.0, p, p, p, p, None, 0, None) == E
+    assert lib.topk_sample_bf16(p, 1, 8, 4, 2, 1, 0.0, p, p, p, p, None, 0, None) == E
+    assert lib.topk_sample_bf16(p, 1, 8, 4, 2, 1, 1.0, None, p, p, p, None, 0, None) == E
+    assert lib.topk_sample_bf16(None, 1, 8, 4, 2, 1, 1.0, p, p, p, p, None, 0, None) == E
 
 
 def test_selftest_rejects_bad_limits_on_host(lib):

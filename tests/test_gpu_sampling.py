@@ -93,3 +93,23 @@ def test_sample_rows_larger_k(oracle_mod):
     otok, margin = oracle_mod.sample_rows(v.cpu().numpy(), i.cpu().numpy(), 0.25,
                                           u.numpy().astype(np.float64))
     _check(tok.cpu().numpy(), otok, margin)
+
+
+@pytest.mark.parametrize("rows,n,k,b,kb,T", [
+    (64, 131072, 50, 512, 1, 1.0),
+    (16, 128256, 256, 256, 1, 0.7),
+    (8, 65536, 64, 512, 4, 1.0),   # the 16-warp k_b > 2 kernel with the draw
+])
+def test_topk_sample_bf16_vs_oracle(oracle_mod, rows, n, k, b, kb, T):
+    """bf16 logits: the selection equals the oracle's on the exactly widened
+    values, and the draw agrees away from CDF boundaries."""
+    x = inputs.vocab_logits(rows, n, 0x5B + n + k).to(torch.bfloat16)
+    u = _uniforms(rows, k + 1)
+    tok, v, i = atk.topk_sample(x.to(DEV), k, b, kb, T, u.to(DEV))
+    assert v.dtype == torch.bfloat16
+    ov, oi = oracle_mod.bucketed(x.float().numpy(), k, b, kb)
+    assert np.array_equal(i.cpu().numpy(), oi)
+    got = v.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, (ov.view(np.uint32) >> 16).astype(np.uint16))
+    otok, margin = oracle_mod.sample_rows(ov, oi, T, u.numpy().astype(np.float64))
+    _check(tok.cpu().numpy(), otok, margin)
