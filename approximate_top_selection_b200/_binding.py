@@ -98,22 +98,35 @@ def _stream_handle(stream, device_index: int) -> int:
 
 class _OnDevice:
     """Makes the tensor's device current for a call, switching only when it
-    is not current already (a device context costs microseconds per call)."""
+    is not current already (a device context costs microseconds per call).
 
-    __slots__ = ("index", "prev")
+    With an explicit `stream`, that stream is also made torch's current stream
+    for the call, so the outputs and the zero-filled workspace the binding
+    allocates are created (and the workspace zeroed) on the stream the kernel
+    runs on: the kernel is ordered after the fill, and the caching allocator
+    recycles those blocks only for later work of that same stream."""
 
-    def __init__(self, device: torch.device):
+    __slots__ = ("index", "prev", "stream", "stream_ctx")
+
+    def __init__(self, device: torch.device, stream=None):
         self.index = device.index if device.index is not None else torch.cuda.current_device()
         self.prev = None
+        self.stream = stream
+        self.stream_ctx = None
 
     def __enter__(self):
         cur = torch.cuda.current_device()
         if cur != self.index:
             self.prev = cur
             torch.cuda.set_device(self.index)
+        if self.stream is not None:
+            self.stream_ctx = torch.cuda.stream(self.stream)
+            self.stream_ctx.__enter__()
         return self
 
     def __exit__(self, *exc):
+        if self.stream_ctx is not None:
+            self.stream_ctx.__exit__(*exc)
         if self.prev is not None:
             torch.cuda.set_device(self.prev)
         return False
@@ -185,7 +198,7 @@ def topk_bucketed(scores: torch.Tensor, k: int, b: int, kb: int, *, out_vals=Non
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with _OnDevice(scores.device) as on:
+    with _OnDevice(scores.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         need = topk_workspace_bytes(TOPK_OP_BUCKETED, rows, n, k, b, kb)
@@ -205,7 +218,7 @@ def topk_bucketed_bf16(scores: torch.Tensor, k: int, b: int, kb: int, *, out_val
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with _OnDevice(scores.device) as on:
+    with _OnDevice(scores.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx, torch.bfloat16)
         need = topk_workspace_bytes(TOPK_OP_BUCKETED_BF16, rows, n, k, b, kb)
@@ -229,7 +242,7 @@ def topk_bucketed_noalloc(scores: torch.Tensor, k: int, b: int, kb: int, *, out_
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with _OnDevice(scores.device) as on:
+    with _OnDevice(scores.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         st = lib.topk_bucketed_noalloc(scores.data_ptr(), rows, n, k, b, kb, out_vals.data_ptr(),
@@ -245,7 +258,7 @@ def topk_exact(scores: torch.Tensor, k: int, *, out_vals=None, out_idx=None, str
     if scores.dim() != 2:
         raise ValueError("scores must be [rows, n]")
     rows, n = scores.shape
-    with _OnDevice(scores.device) as on:
+    with _OnDevice(scores.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, scores.device, out_vals, out_idx)
         st = lib.topk_exact(scores.data_ptr(), rows, n, k, out_vals.data_ptr(),
@@ -277,7 +290,7 @@ def topk_bucketed_merge(vals: torch.Tensor, idx: torch.Tensor, n_total: int, k: 
     if len(offs) != parts:
         raise ValueError("part_offsets needs one entry per part")
     c_offs = (ctypes.c_int64 * parts)(*offs)
-    with _OnDevice(vals.device) as on:
+    with _OnDevice(vals.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, vals.device, out_vals, out_idx)
         st = lib.topk_bucketed_merge(vals.data_ptr(), idx.data_ptr(), parts, rows, m, c_offs,
@@ -309,7 +322,7 @@ def score_rerank(q: torch.Tensor, K: torch.Tensor, cand_idx: torch.Tensor, k: in
         n, kstride = K.shape[0], 0
     else:
         raise ValueError("K must be [rows, n, d] or [n, d]")
-    with _OnDevice(q.device) as on:
+    with _OnDevice(q.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
         scores = torch.empty(rows, c, dtype=torch.float32, device=q.device) if return_scores else None
@@ -331,7 +344,7 @@ def topk_sample_rows(vals: torch.Tensor, idx: torch.Tensor, temperature: float, 
     if vals.dim() != 2 or tuple(idx.shape) != tuple(vals.shape) or u.numel() != vals.shape[0]:
         raise ValueError("vals, idx must be [rows, k] and u [rows]")
     rows, k = vals.shape
-    with _OnDevice(vals.device) as on:
+    with _OnDevice(vals.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         if out_token is None:
             out_token = torch.empty(rows, dtype=torch.int32, device=vals.device)
@@ -354,7 +367,7 @@ def topk_sample(logits: torch.Tensor, k: int, b: int, kb: int, temperature: floa
     if logits.dim() != 2 or u.numel() != logits.shape[0]:
         raise ValueError("logits must be [rows, n] and u [rows]")
     rows, n = logits.shape
-    with _OnDevice(logits.device) as on:
+    with _OnDevice(logits.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, logits.device, out_vals, out_idx,
                                      dtype=torch.bfloat16 if bf16 else torch.float32)
@@ -397,7 +410,7 @@ def score_topk(q: torch.Tensor, K: torch.Tensor, k: int, b: int, kb: int, *,
         raise ValueError("K must be [rows, n, d] or [n, d]")
     if K.shape[-1] != d:
         raise ValueError("q and K disagree on d")
-    with _OnDevice(q.device) as on:
+    with _OnDevice(q.device, stream) as on:
         sh = _stream_handle(stream, on.index)
         out_vals, out_idx = _outputs(rows, k, q.device, out_vals, out_idx)
         scores = torch.empty(rows, n, dtype=torch.float32, device=q.device) if return_scores else None
@@ -418,7 +431,7 @@ def topk_selftest_wait_timeout(limit_ns: int = 1_000_000, stream=None) -> None:
     """Queue a bounded wait that is sure to expire (see the header); the next
     topk_device_status() then reports the expiry."""
     lib = load_library()
-    with _OnDevice(torch.device("cuda", torch.cuda.current_device())) as on:
+    with _OnDevice(torch.device("cuda", torch.cuda.current_device()), stream) as on:
         _check(lib.topk_selftest_wait_timeout(int(limit_ns), _stream_handle(stream, on.index)),
                "topk_selftest_wait_timeout")
 

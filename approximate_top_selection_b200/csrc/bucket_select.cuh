@@ -239,8 +239,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA can go away.
-        for (int64_t u = (t > stages ? t - stages : 0); u < t; ++u)
-          mbar_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), 100000000ull);
+        drain_copies(full, stages, t > stages ? t - stages : 0, t);
       }
     }
     return;
@@ -474,8 +473,7 @@ __global__ void __launch_bounds__(kWideThreads, 2) bucket_select_wide(SelectArgs
         }
       }
       if (*abort_flag) {
-        for (int64_t u = (t > stages ? t - stages : 0); u < t; ++u)
-          mbar_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), 100000000ull);
+        drain_copies(full, stages, t > stages ? t - stages : 0, t);
       }
     }
     return;

@@ -159,6 +159,34 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parit
   return true;
 }
 
+// Device status bit of a drain that expired (TOPK_DEV_DRAIN_TIMEOUT).
+constexpr int kDevDrainTimeout = 4;
+
+// One wait of the drain that follows an abort: all waits of one drain share a
+// single deadline, kWaitLimitNs after `start`.  On expiry records
+// TOPK_DEV_DRAIN_TIMEOUT and returns false.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity,
+                                           unsigned long long start) {
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - start > kWaitLimitNs) {
+      atomicOr(&g_device_status, kDevDrainTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// After an abort, the producer waits until the bulk copies it already issued
+// -- tiles [t0, t1) of a ring of `stages` stages with full barriers `full` --
+// have landed, so that the CTA never exits while a copy still writes into its
+// shared memory.  If even that drain runs out of time, the status says so and
+// the CTA exits anyway: the context is then to be treated as unusable.
+__device__ __forceinline__ void drain_copies(uint64_t* full, int stages, int64_t t0, int64_t t1) {
+  const unsigned long long start = global_ns();
+  for (int64_t u = t0; u < t1; ++u)
+    if (!drain_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), start)) return;
+}
+
 // Barrier over the first `nthreads` threads of the CTA (named barrier 1), so a
 // producer warp outside that group never has to take part.
 __device__ __forceinline__ void group_sync(int nthreads) {

@@ -124,8 +124,7 @@ __global__ void __launch_bounds__(kScorePipeThreads, 2)
         }
       }
       if (*abort_flag) {
-        for (int64_t u = (t > stages ? t - stages : 0); u < t; ++u)
-          mbar_wait(full + (u % stages), static_cast<uint32_t>((u / stages) & 1), 100000000ull);
+        drain_copies(full, stages, t > stages ? t - stages : 0, t);
       }
     }
     return;

@@ -16,10 +16,12 @@
 // (t0 + c%32)*b + 8g + c/32: each 32-column TMEM load is one bucket's 32
 // stripes, so an epilogue warp owns whole buckets and needs no merge.
 //
-// Warp roles (320 threads): warp 0 issues TMA loads (Q tile once per unit, key
-// stages through a ring), warp 1 owns TMEM (512 columns = two 128x256 fp32
-// accumulators) and issues the MMAs from one thread, warps 2..9 drain TMEM
-// (tcgen05.ld) and update the queues: H warps per TMEM lane quarter, each
+// Warp roles (576 threads for k_b <= 2, 320 for k_b > 2): warp 0 issues TMA
+// loads (Q tile once per unit, key stages through a ring), warp 1 owns TMEM
+// (512 columns = two 128x256 fp32 accumulators) and issues the MMAs from one
+// thread, and the epilogue warps -- 2..17 (16 warps) for k_b <= 2, 2..9 (8
+// warps, more registers per thread for the longer queues) for k_b > 2 -- drain
+// TMEM (tcgen05.ld) and update the queues: H warps per TMEM lane quarter, each
 // owning 8/H buckets (H = 4 for k_b <= 2, 2 for larger queues).  Per-unit
 // results (top-k_b per bucket) go to the workspace; umma_finish runs Stage 2.
 //
@@ -332,10 +334,12 @@ __global__ void __launch_bounds__(umma_threads(KB), 1)
       }
       if (*abort_flag) {
         // Let the copies already issued land before the CTA can go away.
-        for (int64_t x = (bt > kUmmaStages ? bt - kUmmaStages : 0); x < bt; ++x)
-          mbar_wait(full_b + (x % kUmmaStages), static_cast<uint32_t>((x / kUmmaStages) & 1),
-                    100000000ull);
-        if (iu > 0) mbar_wait(a_full, static_cast<uint32_t>((iu - 1) & 1), 100000000ull);
+        const unsigned long long start = global_ns();
+        bool drained = true;
+        for (int64_t x = (bt > kUmmaStages ? bt - kUmmaStages : 0); drained && x < bt; ++x)
+          drained = drain_wait(full_b + (x % kUmmaStages),
+                               static_cast<uint32_t>((x / kUmmaStages) & 1), start);
+        if (drained && iu > 0) drain_wait(a_full, static_cast<uint32_t>((iu - 1) & 1), start);
       }
     }
   } else if (warp == 1) {

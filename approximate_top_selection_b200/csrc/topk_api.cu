@@ -563,22 +563,38 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[TOPK_NOALLOC_SC
 
 struct ScratchAddr {
   bool init = false;
+  CUcontext ctx = nullptr;  // the context the address belongs to
   void* ptr = nullptr;
 };
 ScratchAddr g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mu;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
 
-// Device address of g_noalloc_scratch on the current device (looked up once).
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device and context: after a device reset the runtime creates a new
+// context in which the buffer has a new address, so the lookup is redone.
 int noalloc_scratch_ptr(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TOPK_ECUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_ctx_current) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || fn == nullptr)
+      return TOPK_ECUDA;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  CUcontext ctx = nullptr;  // null until the runtime has bound the device's context
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return TOPK_ECUDA;
   ScratchAddr& s = g_scratch_addr[dev];
-  if (!s.init) {
+  if (!s.init || ctx == nullptr || s.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return TOPK_ECUDA;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return TOPK_ECUDA;
     s.ptr = p;
+    s.ctx = ctx;
     s.init = true;
   }
   *out = s.ptr;

@@ -16,9 +16,17 @@ top-k (with Eq. (1) of "Approximate Top-k for Increased Parallelism" beside it)
 ride along.  Timing protocol after that paper's benchmark appendix: warm-up
 launches, then device-side CUDA events around K steps.
 
-Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
-inputs (rows are independent; no collective on the data path); the time is the
-maximum over ranks and `value` counts the bytes of all ranks (weak scaling).
+Multi-GPU (`--gpus N`, one rank per GPU; started as one process it relaunches
+itself under torch.distributed.run): every rank runs the same per-GPU workload
+on its own inputs (rows are independent; no collective on the data path),
+except `vocab-split`, whose rows are cut by columns across the ranks and merged
+after one all-gather of the candidate pairs; the time is the maximum over
+ranks and `value` counts the bytes of all ranks (weak scaling).
+
+A one-GPU run also carries `sweep`: every score-row workload (vocabulary and
+the long-context b x k_b grid, fp32 and bf16) and the fused link and re-rank
+workloads, each timed on its own from CUDA-graph replays, with its roofline
+fraction and clock record.
 """
 from __future__ import annotations
 
@@ -65,8 +73,21 @@ for _b in (128, 256, 512):
 # from the softmax (T = 1) of the selected logits
 CONFIGS["vocab-sample"] = dict(CONFIGS["vocab"], sample=1.0)
 # bfloat16 score rows (the page's Fig. 10 repeats its configurations in bf16)
-for _name in ("vocab", "long-b128-kb1", "long-b256-kb2", "long-b512-kb4"):
+for _name in ["vocab"] + ["long-b%d-kb%d" % (b, kb) for b in (128, 256, 512) for kb in (1, 2, 4)]:
     CONFIGS[_name + "-bf16"] = dict(CONFIGS[_name], dtype="bf16")
+# vocabulary-parallel rows: every rank holds 131072 columns of each of the 256
+# rows (a row of world x 131072 logits in all), selects on its slice,
+# all-gathers the k (value, index) pairs per row and merges them by global
+# index (sharded.split_row_topk).  Per-rank work is fixed: weak scaling.
+CONFIGS["vocab-split"] = dict(CONFIGS["vocab"], kind="split")
+
+L2_BYTES = 126 * 2 ** 20
+
+# The cells of the score-row sweep that rides along with the default line.
+SWEEP = (["vocab", "vocab-bf16", "vocab-sample"]
+         + ["long-b%d-kb%d%s" % (b, kb, t) for t in ("", "-bf16") for b in (128, 256, 512)
+            for kb in (1, 2, 4)]
+         + ["link", "decode-rerank"])
 
 
 def _peaks():
@@ -144,10 +165,11 @@ class ClockSampler:
 class Workload:
     """Resident device inputs for one config, plus the step function."""
 
-    def __init__(self, name: str, device, seed_offset: int = 0):
+    def __init__(self, name: str, device, seed_offset: int = 0, rank: int = 0, world: int = 1):
         from approximate_top_selection_b200 import inputs
 
         self.name, self.cfg, self.device = name, CONFIGS[name], device
+        self.rank, self.world = rank, world
         c = self.cfg
         seed = inputs.SEEDS[name.split("-")[0]] + seed_offset
         if c["kind"] == "rerank":
@@ -188,7 +210,6 @@ class Workload:
             self.in_bytes += self.rows * 4
             self.out_bytes += self.rows * 4
         self.bytes = self.in_bytes + self.out_bytes
-        self.larger_than_l2 = self.in_bytes > 126 * 2 ** 20
 
     def step(self, stream=None):
         import approximate_top_selection_b200 as atk
@@ -200,7 +221,18 @@ class Workload:
             return atk.score_rerank(self.q, self.K, self.cand, c["k"], stream=stream)
         if c.get("sample"):
             return atk.topk_sample(self.x, c["k"], c["b"], c["kb"], c["sample"], self.u, stream=stream)
+        if c["kind"] == "split":
+            return self.split_step(self.x)
         return atk.topk_bucketed(self.x, c["k"], c["b"], c["kb"], stream=stream)
+
+    def split_step(self, x):
+        """This rank's slice of the rows: local selection, all-gather of the
+        candidate pairs, merge by global index."""
+        from approximate_top_selection_b200 import sharded
+
+        c = self.cfg
+        return sharded.split_row_topk(x, self.rank * c["n"], self.world * c["n"], c["k"], c["b"],
+                                      c["kb"], offsets=[r * c["n"] for r in range(self.world)])
 
     def oracle_step(self, rows: int):
         """A callable doing this workload's step with the oracle on its first `rows` rows."""
@@ -247,14 +279,31 @@ def _kernel_name(cfg) -> str:
 
 
 def _launches_per_step(cfg) -> int:
-    # the tensor-core path adds a Stage-2 kernel; the sampling draw runs inside
-    # the selection kernel
-    return 2 if _uses_tensor_cores(cfg) else 1
+    # the tensor-core path adds a Stage-2 kernel, the row split a merge kernel;
+    # the sampling draw runs inside the selection kernel
+    return 2 if _uses_tensor_cores(cfg) or cfg["kind"] == "split" else 1
 
 
 def _rotations(w: Workload) -> int:
-    """Input copies needed so that consecutive steps do not hit in L2."""
-    return 1 if w.larger_than_l2 else max(2, math.ceil(3 * 126 * 2 ** 20 / w.in_bytes))
+    """Input copies cycled through so that every step reads its input from
+    HBM: one copy when the input is at least twice the L2, else enough copies
+    to span three L2s."""
+    if w.in_bytes >= 2 * L2_BYTES:
+        return 1
+    return max(2, math.ceil(3 * L2_BYTES / w.in_bytes))
+
+
+def _l2_note(w: Workload, nrot: int) -> str:
+    if nrot == 1:
+        return "inputs larger than twice the L2"
+    return "%d rotating input copies (%.0f MiB) defeat L2" % (nrot, nrot * w.in_bytes / 2 ** 20)
+
+
+def _config(w: Workload, nrot: int, graph: bool) -> dict:
+    """The `config` object of a line: the workload, how L2 is defeated and
+    how steps are launched (the same object for both arms)."""
+    return dict(w.describe(), l2=_l2_note(w, nrot),
+                launch="cuda-graph replay" if graph else "eager")
 
 
 def _time_ms(fn, steps: int, warmup: int = 3) -> float:
@@ -278,7 +327,7 @@ def exact_context(w: Workload, ms_bucketed: float, steps: int = 20):
 
     c = w.cfg
     out = {"bucketed_ms": ms_bucketed}
-    if c["kind"] == "select":
+    if c["kind"] in ("select", "split"):
         x = w.x.float() if w.x.dtype != torch.float32 else w.x
         out["exact_topk_ms"] = _time_ms(lambda: atk.topk_exact(x, c["k"]), steps)
         out["torch_topk_ms"] = _time_ms(lambda: torch.topk(w.x, c["k"], dim=1), steps)
@@ -358,17 +407,25 @@ def cpu_baseline(w: Workload, budget_s: float = 10.0):
 
 # ---------------------------------------------------------------- runs
 def setup_dist(args):
+    """One process per GPU: the NCCL process group from torchrun's variables.
+    A row-split workload on one GPU still runs its collective, in a
+    one-rank group."""
+    import datetime
+
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    timeout = datetime.timedelta(seconds=120)
     if world > 1:
-        import datetime
-
         torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+        torch.distributed.init_process_group("nccl", timeout=timeout,
                                              device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
+        if CONFIGS[args.config]["kind"] == "split":
+            torch.distributed.init_process_group("nccl", store=torch.distributed.HashStore(),
+                                                 rank=0, world_size=1, timeout=timeout,
+                                                 device_id=torch.device("cuda", 0))
     return world, rank, local
 
 
@@ -398,9 +455,10 @@ def run_ours(args, world, rank, local):
 
     atk.load_library()
     dev = torch.device("cuda", local)
-    w = Workload(args.config, dev, seed_offset=rank)
+    w = Workload(args.config, dev, seed_offset=rank, rank=rank, world=world)
     nrot = _rotations(w)
-    extra = [Workload(args.config, dev, seed_offset=rank + 101 * (j + 1)) for j in range(nrot - 1)]
+    extra = [Workload(args.config, dev, seed_offset=rank + 101 * (j + 1), rank=rank, world=world)
+             for j in range(nrot - 1)]
     works = [w] + extra
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -452,13 +510,10 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16" if w.cfg.get("dtype") == "bf16" else "f32",
         "data": "synthetic (seeded; shapes of the pages' workloads)",
-        "config": dict(w.describe(), l2="inputs larger than L2" if nrot == 1 else
-                       "%d rotating input copies (%.0f MiB) defeat L2" %
-                       (nrot, nrot * w.in_bytes / 2 ** 20),
-                       launch="cuda-graph replay" if args.graph else "eager"),
+        "config": _config(w, nrot, args.graph),
         "rows_per_s": w.rows * world / (ms_step * 1e-3),
         "gpu_launches": args.steps * _launches_per_step(w.cfg),
-        "roofline": _roofline(w, ms_step, achieved, hbm, peak_src),
+        "roofline": _roofline(w, ms_step, achieved, hbm, peak_src, ms_step * args.steps * 1e-3),
         "clocks": clk.summary(),
     }
     if not args.no_recall:
@@ -469,7 +524,76 @@ def run_ours(args, world, rank, local):
         line["e2e"] = e2e(w, args, world)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w)
+    if world == 1 and not args.no_sweep:
+        del run, works, extra, w
+        if args.graph:
+            del graphs, g
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        line["sweep"] = sweep(dev, local)
     return line
+
+
+def _graph_of_steps(works, reps: int):
+    """One CUDA graph holding `reps` passes over the input copies (one step
+    per copy): a replay launches len(works) * reps steps with no host work."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for wk in works:  # workspace and kernel set-up on the capturing stream
+            wk.step()
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(reps):
+            for wk in works:
+                wk.step()
+    return g
+
+
+def sweep_cell(name: str, dev, local: int, min_region_s: float = 0.25) -> dict:
+    """One workload timed alone: CUDA-graph replays of back-to-back steps over
+    rotating input copies, CUDA events around the replays, clocks sampled
+    meanwhile."""
+    w = Workload(name, dev)
+    nrot = _rotations(w)
+    works = [w] + [Workload(name, dev, seed_offset=101 * (j + 1)) for j in range(nrot - 1)]
+    reps = max(1, 24 // nrot)
+    g = _graph_of_steps(works, reps)
+    per_replay = nrot * reps
+    for _ in range(3):
+        g.replay()
+    est = _time_ms(g.replay, 3, warmup=0) / per_replay
+    replays = max(3, math.ceil(min_region_s * 1e3 / (est * per_replay)))
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(replays):
+            g.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    steps = replays * per_replay
+    ms = ev0.elapsed_time(ev1) / steps
+    hbm, _, peak_src = _peaks()
+    gbs = w.bytes / (ms * 1e-3) / 1e9
+    roof = _roofline(w, ms, gbs, hbm, peak_src, ms * steps * 1e-3)
+    out = {"ms_per_step": ms, "GB/s": gbs, "rows_per_s": w.rows / (ms * 1e-3),
+           "bound": roof["bound"], "achieved": roof["achieved"], "unit": roof["unit"],
+           "frac": roof["frac"], "kernel": roof["kernel"], "steps": steps,
+           "l2": _l2_note(w, nrot), "clocks": clk.summary()}
+    del g, works, w
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def sweep(dev, local: int) -> dict:
+    """Every score-row cell (vocab, fp32 and bf16; the long-context b x k_b
+    grid, fp32 and bf16) and the fused link and re-rank workloads, each timed
+    on its own."""
+    return {name: sweep_cell(name, dev, local) for name in SWEEP}
 
 
 # Device sources of each timed kernel: a traffic figure stays valid while these
@@ -510,12 +634,13 @@ def _traffic(workload: str):
     return None
 
 
-def _roofline(w: Workload, ms_step: float, achieved_gbs: float, hbm: float, peak_src: str):
+def _roofline(w: Workload, ms_step: float, achieved_gbs: float, hbm: float, peak_src: str,
+              region_s: float):
     c = w.cfg
     if _uses_tensor_cores(c):
         flops = 2.0 * w.rows * c["n"] * c["d"]
         tf = flops / (ms_step * 1e-3) / 1e12
-        peak, src = _tensor_peak()
+        peak, src = _tensor_peak(region_s)
         return {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
                 "frac": tf / peak, "traffic": _traffic(w.name), "kernel": _kernel_name(c),
                 "flops_per_step": flops, "peak_source": src}
@@ -524,16 +649,21 @@ def _roofline(w: Workload, ms_step: float, achieved_gbs: float, hbm: float, peak
             "peak_source": peak_src + " hbm_gbs"}
 
 
-def _tensor_peak():
-    """Dense bf16 peak for a GEMM timed inside a long loop: the sustained figure."""
+SUSTAINED_REGION_S = 2.0  # timed regions at least this long compare with the sustained peak
+
+
+def _tensor_peak(region_s: float):
+    """Dense bf16 peak: the burst figure for a timed region shorter than
+    SUSTAINED_REGION_S, the sustained (power-capped) one for a longer one."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    long_region = region_s >= SUSTAINED_REGION_S
     if os.path.exists(path):
         with open(path) as f:
             p = json.load(f)
-        if "bf16_tflops_sustained" in p:
+        if long_region and "bf16_tflops_sustained" in p:
             return float(p["bf16_tflops_sustained"]), "measured bf16_tflops_sustained"
         return float(p["bf16_tflops"]), "measured bf16_tflops"
-    return 1400.0, "fallback (sustained)"
+    return (1400.0, "fallback (sustained)") if long_region else (1590.0, "fallback (burst)")
 
 
 def e2e(w: Workload, args, world):
@@ -586,6 +716,9 @@ def e2e(w: Workload, args, world):
             du.copy_(hu, non_blocking=True)
             t, v, i = atk.topk_sample(dx, c["k"], c["b"], c["kb"], c["sample"], du)
             ht.copy_(t, non_blocking=True)
+        elif c["kind"] == "split":
+            dx.copy_(hx, non_blocking=True)
+            v, i = w.split_step(dx)
         else:
             dx.copy_(hx, non_blocking=True)
             v, i = atk.topk_bucketed(dx, c["k"], c["b"], c["kb"])
@@ -606,8 +739,13 @@ def e2e(w: Workload, args, world):
             "ms_per_step": ms, "steps": steps}
 
 
+REFERENCE_BUDGET_S = 60.0  # host seconds for the reference arm's warm-up and timed steps
+
+
 def run_reference(args, world, rank, local):
-    """The oracle on the host cores: each step is a bounded row sample."""
+    """The oracle on the host cores, as it stands: every step is a bounded
+    row sample of the same workload, sized so that the W warm-up and K timed
+    steps take about REFERENCE_BUDGET_S together."""
     import oracle
 
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
@@ -615,25 +753,24 @@ def run_reference(args, world, rank, local):
     oracle.build()
     threads = oracle.max_threads()
     oracle.set_threads(threads)
-    c = w.cfg
-    # sample size: about 1 s of oracle work per step
     probe = cpu_baseline(w, budget_s=1.0)
-    rows = max(1, min(w.rows, int(probe["rows_per_s"] * 1.0)))
+    per_step_s = min(1.0, max(0.02, REFERENCE_BUDGET_S / (args.steps + args.warmup)))
+    rows = max(1, min(w.rows, int(probe["rows_per_s"] * per_step_s)))
     step = w.oracle_step(rows)
-    for _ in range(min(args.warmup, 3)):
+    for _ in range(args.warmup):
         step()
-    steps = max(1, min(args.steps, 20))
     t0 = time.perf_counter()
-    for _ in range(steps):
+    for _ in range(args.steps):
         step()
-    dt = (time.perf_counter() - t0) / steps
+    dt = (time.perf_counter() - t0) / args.steps
     per_row = w.bytes / w.rows
     value = rows * per_row / dt / 1e9
     sample = "%d of %d rows of the %s workload per step" % (rows, w.rows, w.name)
-    return {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
-            "warmup": min(args.warmup, 3), "ms_per_step": dt * 1e3, "higher_is_better": True,
+    return {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate / f32 select",
-            "data": "synthetic", "impl": "reference", "config": w.describe(),
+            "data": "synthetic (seeded; shapes of the pages' workloads)", "impl": "reference",
+            "config": _config(w, _rotations(w), args.graph),
             "rows_per_s": rows / dt,
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
@@ -656,11 +793,21 @@ def main():
                     help="time CUDA-graph replays of the step instead of eager launches")
     ap.add_argument("--context", action="store_true",
                     help="also time exact top-k (this library and torch.topk) on the same input")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-workload sweep that rides along with a one-GPU line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.graph and CONFIGS[args.config]["kind"] == "split":
+        ap.error("the row-split workload holds collectives: it is timed eagerly")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        relaunch_with_torchrun(args.gpus)  # does not return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        ap.error("--gpus %d but %d ranks were launched (WORLD_SIZE)" % (args.gpus, world))
     if args.impl == "reference":
         if rank != 0:
             return
@@ -671,8 +818,24 @@ def main():
     line = run_ours(args, world, rank, local)
     if rank == 0:
         print(json.dumps(line))
-    if world > 1:
+    if torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
+
+
+def relaunch_with_torchrun(n: int) -> None:
+    """`bench.py --gpus N` started as a single process: run it again as N
+    ranks, one per GPU, under torch.distributed.run on this node."""
+    import socket
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    sys.stdout.flush()
+    os.execv(sys.executable, cmd)
 
 
 if __name__ == "__main__":

@@ -217,7 +217,9 @@ int score_topk(const uint16_t *q_dev, int64_t rows, int d, const uint16_t *K_dev
  *     cudaFree or library allocator.
  *   - The first call on a device looks up that device's address of the buffer
  *     (with the device current); make that first call before any stream
- *     capture begins on the device.
+ *     capture begins on the device.  The address is kept per device and
+ *     context: after a device reset the first call in the new context looks
+ *     it up again, with the same rule on capture.
  *   - A call whose scratch need exceeds the buffer returns TOPK_ESCRATCH and
  *     queues nothing; topk_workspace_bytes(TOPK_OP_BUCKETED, ...) tells the
  *     need in advance.
@@ -251,6 +253,10 @@ int topk_device_status(int *status_out);
 
 #define TOPK_DEV_WAIT_TIMEOUT 1 /* a bulk-copy wait in a streaming kernel expired */
 #define TOPK_DEV_BAD_INDEX 2    /* topk_bucketed_merge or score_rerank skipped an index out of range */
+#define TOPK_DEV_DRAIN_TIMEOUT 4 /* after an expired wait, the kernel's wait for its own bulk copies
+                                    still in flight expired too: the kernel returned while a copy
+                                    may still have been writing to its shared memory, so the
+                                    context must be treated as unusable (reset or exit) */
 
 #ifdef __cplusplus
 }

@@ -50,14 +50,40 @@ def test_launches_per_step():
 class _W:
     def __init__(self, in_bytes):
         self.in_bytes = in_bytes
-        self.larger_than_l2 = in_bytes > 126 * 2 ** 20
 
 
 def test_rotations_defeat_l2():
+    """Inputs under twice the L2 (the 128 MiB score rows among them) rotate
+    over copies spanning at least three L2s; larger inputs stream as they are."""
     assert bench._rotations(_W(4 << 30)) == 1
-    for b in (1 << 17, 64 << 20, 120 << 20):
+    assert bench._rotations(_W(2 * bench.L2_BYTES)) == 1
+    for b in (1 << 17, 64 << 20, 120 << 20, 128 << 20, 2 * bench.L2_BYTES - 1):
         n = bench._rotations(_W(b))
-        assert n >= 2 and n * b >= 3 * 126 * 2 ** 20
+        assert n >= 2 and n * b >= 3 * bench.L2_BYTES
+
+
+def test_tensor_peak_burst_or_sustained():
+    """A timed region shorter than a couple of seconds compares with the burst
+    GEMM peak, a longer one with the sustained (power-capped) figure."""
+    short, src_s = bench._tensor_peak(0.05)
+    long_, src_l = bench._tensor_peak(10.0)
+    assert "sustained" not in src_s and short >= long_
+    assert "sustained" in src_l
+
+
+def test_sweep_cells_exist():
+    for name in bench.SWEEP:
+        assert name in bench.CONFIGS, name
+    for b in (128, 256, 512):
+        for kb in (1, 2, 4):
+            assert "long-b%d-kb%d" % (b, kb) in bench.SWEEP
+            assert "long-b%d-kb%d-bf16" % (b, kb) in bench.SWEEP
+    assert {"vocab", "vocab-bf16"} <= set(bench.SWEEP)
+
+
+def test_split_workload_launches():
+    assert bench._launches_per_step(bench.CONFIGS["vocab-split"]) == 2
+    assert bench._kernel_name(bench.CONFIGS["vocab-split"]) == "bucket_select_tma"
 
 
 def test_job_throughput_is_weak_scaling():

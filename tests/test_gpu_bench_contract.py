@@ -8,6 +8,8 @@ import sys
 
 import pytest
 
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
 pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -26,7 +28,7 @@ def _run(*args):
 
 @pytest.mark.parametrize("extra", [[], ["--graph"]])
 def test_bench_line(extra):
-    d = _run("--config", "tiny", "--steps", "20", "--warmup", "3", "--no-cpu", *extra)
+    d = _run("--config", "tiny", "--steps", "20", "--warmup", "3", "--no-cpu", "--no-sweep", *extra)
     assert KEYS <= set(d)
     assert d["value"] > 0 and d["n_gpus"] == 1 and d["steps"] == 20 and d["warmup"] == 3
     assert d["config"]["workload"] == "tiny"
@@ -43,3 +45,31 @@ def test_reference_line():
     assert d["impl"] == "reference" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["steps"] == 2 and d["warmup"] == 3
+    ours = _run("--config", "tiny", "--steps", "2", "--warmup", "3", "--no-cpu", "--no-sweep",
+                "--no-e2e")
+    assert d["config"] == ours["config"]
+    assert (d["metric"], d["unit"], d["higher_is_better"]) == \
+        (ours["metric"], ours["unit"], ours["higher_is_better"])
+
+
+def test_default_line_carries_the_sweep():
+    """The default workload's line, with the sweep of every score-row cell
+    (fp32 and bf16) and the fused workloads, each with its own timing."""
+    d = _run("--steps", "5", "--warmup", "3", "--no-cpu", "--no-e2e", "--no-recall")
+    assert d["config"]["workload"] == "decode"
+    sw = d["sweep"]
+    import bench
+    assert set(sw) == set(bench.SWEEP)
+    for name, cell in sw.items():
+        assert cell["ms_per_step"] > 0 and 0 < cell["frac"] < 1.5, name
+        assert cell["bound"] in ("hbm", "tensor"), name
+
+
+def test_split_workload_one_gpu():
+    """The vocabulary-parallel workload in a one-rank group: selection on the
+    slice, the NCCL all-gather, the merge kernel; two launches per step."""
+    d = _run("--config", "vocab-split", "--steps", "10", "--warmup", "3", "--no-cpu",
+             "--no-sweep")
+    assert d["config"]["workload"] == "vocab-split" and d["gpu_launches"] == 20
+    assert d["value"] > 0 and d["recall"]["mean"] > 0.9

@@ -281,10 +281,28 @@ def test_score_long_rows_split(oracle_mod):
     check_scores(q.to(DEV), K.to(DEV), 512, 256, 2, oracle_mod)
 
 
+def _cta_edge_rows(rows: int, n: int, ctas: int, extra: int, seed: int) -> list:
+    """Sampled rows: the rows holding the first and the last element of CTA
+    ranges when rows*n elements are cut into `ctas` equal ranges (the
+    streaming kernels' split), plus `extra` rows drawn at random."""
+    E = rows * n
+    picked = set()
+    for c in range(0, ctas, max(1, ctas // 24)):
+        lo, hi = E * c // ctas, E * (c + 1) // ctas - 1
+        picked.update((lo // n, hi // n))
+    picked.update((0, rows - 1))
+    rng = np.random.default_rng(seed)
+    picked.update(int(r) for r in rng.choice(rows, size=extra, replace=False))
+    return sorted(picked)
+
+
 def test_decode_config_full(oracle_mod):
-    """16 x 32 rows, 32768 keys of d=128: sampled rows against the oracle."""
+    """16 x 32 rows, 32768 keys of d=128: at least 64 sampled rows (the rows at
+    the edges of CTA ranges among them) against the oracle."""
     q, K = inputs.decode_inputs(16, 32, 32768, 128, inputs.SEEDS["decode"], device=DEV)
-    check_scores(q, K, 512, 256, 2, oracle_mod, rows_subset=[0, 1, 100, 255, 256, 400, 511])
+    sub = _cta_edge_rows(512, 32768, 296, 24, 5)
+    assert len(sub) >= 64
+    check_scores(q, K, 512, 256, 2, oracle_mod, rows_subset=sub)
 
 
 # ------------------------------------------------------------------ tensor-core scoring
@@ -315,7 +333,13 @@ def test_link_config_full(oracle_mod):
     """1024 queries x 2^20 entities, d = 256, k = 100, b = 1024, k_b = 1:
     sampled query rows against the fp64 oracle."""
     Q, K = inputs.link_inputs(1024, 1 << 20, 256, inputs.SEEDS["link"], device=DEV)
-    check_scores(Q, K, 100, 1024, 1, oracle_mod, rows_subset=[0, 127, 128, 500, 1023])
+    # the first and last query of each 128-query tile, plus 48 drawn at random
+    edges = {e for t in range(8) for e in (128 * t, 128 * t + 127)}
+    rng = np.random.default_rng(6)
+    rest = [int(r) for r in rng.permutation(1024) if int(r) not in edges][:48]
+    sub = sorted(edges | set(rest))
+    assert len(sub) == 64
+    check_scores(Q, K, 100, 1024, 1, oracle_mod, rows_subset=sub)
 
 
 # ------------------------------------------------------------------ bfloat16 rows

@@ -6,11 +6,11 @@ streams, a framework that forbids allocations it does not account for, a
 plugin that may only allocate at set-up.  For them topk_bucketed_noalloc takes
 only inputs and outputs and keeps its scratch in a static buffer inside the
 library.  These checks call it through the C ABI (ctypes, preallocated
-outputs) and compare it with topk_bucketed, bit for bit, on two calls in a row
-for each shape, including shapes whose rows are split across CTAs (the case
-that needs scratch).  This file is collected last so that a run stopping at
-the first failure has already run every other test; it also passes on its own
-in a fresh process.
+outputs) and compare it, bit for bit, with the CPU oracle and with
+topk_bucketed, on two calls in a row for each shape, including shapes whose
+rows are split across CTAs (the case that needs scratch).  This file is
+collected last so that a run stopping at the first failure has already run
+every other test; it also passes on its own in a fresh process.
 """
 import ctypes
 
@@ -50,17 +50,22 @@ def _noalloc(lib, x, k, b, kb, ov, oi):
 
 
 @pytest.mark.parametrize("rows,n,k,b,kb,kind", SHAPES)
-def test_noalloc_matches_topk_bucketed(rows, n, k, b, kb, kind):
+def test_noalloc_matches_oracle_and_topk_bucketed(rows, n, k, b, kb, kind, oracle_mod):
     if not torch.cuda.is_available():
         pytest.fail("this test needs a CUDA device")
     lib = atk.load_library()
     for call in range(2):  # two calls in a row share (and must clear) the scratch
-        x = _rows(rows, n, kind, 9000 + 17 * call + n).to(DEV)
+        xc = _rows(rows, n, kind, 9000 + 17 * call + n)
+        x = xc.to(DEV)
         ov = torch.empty(rows, k, dtype=torch.float32, device=DEV)
         oi = torch.empty(rows, k, dtype=torch.int32, device=DEV)
         assert _noalloc(lib, x, k, b, kb, ov, oi) == atk.TOPK_OK
         rv, ri = atk.topk_bucketed(x, k, b, kb)
         torch.cuda.synchronize()
+        wv, wi = oracle_mod.bucketed(xc.numpy(), k, b, kb)
+        assert np.array_equal(oi.cpu().numpy(), wi), "indices differ from the oracle (call %d)" % call
+        assert np.array_equal(ov.cpu().numpy().view(np.uint32), wv.view(np.uint32)), \
+            "values differ from the oracle (call %d)" % call
         assert torch.equal(oi, ri), "indices differ from topk_bucketed (call %d)" % call
         assert torch.equal(ov.view(torch.int32), rv.view(torch.int32)), "values differ"
     assert atk.topk_device_status() == 0
