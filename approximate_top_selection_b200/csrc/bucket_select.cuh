@@ -64,20 +64,36 @@ struct SelectArgs {
   SampleTail tail;  // token == nullptr: no sampling tail
 };
 
-// Shared-memory layout of the selection kernels (bytes).
+// Shared-memory layouts of the streaming kernels:
+//  kLayoutSeparate  tile ring, lane buffer (every queue, stored for the
+//                   merge), Stage-2 candidate buffer and barriers side by side.
+//  kLayoutAliased   every CTA streams exactly one piece, so the lane and
+//                   candidate buffers are only needed once the ring has been
+//                   consumed for good: they live inside it, and the ring gets
+//                   their room (more tile stages in flight).
+enum SelectLayout { kLayoutSeparate = 0, kLayoutAliased = 1 };
+
 struct SelectSmem {
   int stages, kb, cand_cap, nl;  // nl: register queues (lanes) per CTA
-  __host__ __device__ size_t ring_bytes() const {
-    return static_cast<size_t>(stages) * kTileBytes;
-  }
+  int layout = kLayoutSeparate;
   __host__ __device__ size_t lane_bytes() const { return static_cast<size_t>(nl) * kb * 8; }
   __host__ __device__ size_t cand_bytes() const {
     return static_cast<size_t>(cand_cap) * 8 + kStage2Extra;
   }
-  __host__ __device__ size_t bar_bytes() const { return 16 * static_cast<size_t>(stages) + 16; }
-  __host__ __device__ size_t total() const {
-    return ring_bytes() + lane_bytes() + cand_bytes() + bar_bytes();
+  __host__ __device__ size_t ring_bytes() const {
+    const size_t r = static_cast<size_t>(stages) * kTileBytes;
+    const size_t lc = lane_bytes() + cand_bytes();
+    return layout == kLayoutAliased && lc > r ? lc : r;
   }
+  __host__ __device__ size_t lane_off() const {
+    return layout == kLayoutAliased ? 0 : ring_bytes();
+  }
+  __host__ __device__ size_t cand_off() const { return lane_off() + lane_bytes(); }
+  __host__ __device__ size_t bar_off() const {
+    return layout == kLayoutAliased ? ring_bytes() : ring_bytes() + lane_bytes() + cand_bytes();
+  }
+  __host__ __device__ size_t bar_bytes() const { return 16 * static_cast<size_t>(stages) + 16; }
+  __host__ __device__ size_t total() const { return bar_off() + bar_bytes(); }
 };
 
 // k_b > 2: one tile (c valid floats at row positions pos_tile ...) for the
@@ -179,18 +195,18 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // (p.tail); without it the sampling code is not compiled in at all.
 template <typename T, int KB, bool SAMPLE = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
-                                                                  int cand_cap) {
+                                                                  int cand_cap, int layout) {
   constexpr int kTileElems = Elem<T>::kPerTile;
   extern __shared__ __align__(128) unsigned char smem[];
-  const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b)};
+  const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b), layout};
   T* ring = reinterpret_cast<T*>(smem);
-  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes() + L.cand_bytes());
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.lane_off());
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.cand_off());
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off());
   uint64_t* empty = full + stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
   int* piece_flag = reinterpret_cast<int*>(empty + stages) + 1;
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(empty + stages) + 2;
 
   const RowSplit& rs = p.rs;
   const int tid = threadIdx.x;
@@ -319,6 +335,16 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     }
     g = pend;
     // Piece done: publish the queues and finish (Stage 2 or cross-CTA merge).
+    // With the lane buffer inside the ring, every consumer must be done with
+    // the ring first (the piece is the CTA's last: no copy is in flight).  An
+    // aborted CTA may still have copies landing there: it stops here, all
+    // consumers together (one thread reads the flag for all of them).
+    if (layout == kLayoutAliased) {
+      group_sync(kThreads);
+      if (tid == 0) *skip_flag = *abort_flag;
+      group_sync(kThreads);
+      if (*skip_flag) break;
+    }
     if (KB <= 2) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
@@ -415,19 +441,19 @@ __device__ __forceinline__ void select_tile_wide(Queues<KB, NQ>& q, const T* til
 
 template <typename T, int KB, int NQ, bool SAMPLE = false>
 __global__ void __launch_bounds__(kWideThreads, 2) bucket_select_wide(SelectArgs<T> p, int stages,
-                                                                   int cand_cap) {
+                                                                   int cand_cap, int layout) {
   constexpr int kTileElems = Elem<T>::kPerTile;
   constexpr int NL = kWideConsumers * NQ;  // register queues (lanes) per CTA
   extern __shared__ __align__(128) unsigned char smem[];
-  const SelectSmem L{stages, KB, cand_cap, NL};
+  const SelectSmem L{stages, KB, cand_cap, NL, layout};
   T* ring = reinterpret_cast<T*>(smem);
-  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.ring_bytes());
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes());
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(smem + L.ring_bytes() + L.lane_bytes() + L.cand_bytes());
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.lane_off());
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.cand_off());
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar_off());
   uint64_t* empty = full + stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
   int* piece_flag = reinterpret_cast<int*>(empty + stages) + 1;
+  volatile int* skip_flag = reinterpret_cast<volatile int*>(empty + stages) + 2;
 
   const RowSplit& rs = p.rs;
   const int tid = threadIdx.x;
@@ -515,6 +541,12 @@ __global__ void __launch_bounds__(kWideThreads, 2) bucket_select_wide(SelectArgs
       done += c;
     }
     g = pend;
+    if (layout == kLayoutAliased) {  // lane buffer inside the ring (see bucket_select_tma)
+      consumer_sync_wide();
+      if (tid == 0) *skip_flag = *abort_flag;
+      consumer_sync_wide();
+      if (*skip_flag) break;
+    }
 #pragma unroll
     for (int v = 0; v < NQ; ++v)
       q.store(v, lanebuf + static_cast<size_t>(tid + kWideConsumers * v) * KB);
@@ -531,8 +563,8 @@ template <typename T, int KB>
 __global__ void __launch_bounds__(kThreads) bucket_select_general(SelectArgs<T> p, int cand_cap) {
   extern __shared__ __align__(128) unsigned char smem[];
   const SelectSmem L{0, KB, cand_cap, kLanes};
-  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.lane_bytes());
+  uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.lane_off());
+  uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.cand_off());
   __shared__ int piece_flag;
 
   const RowSplit& rs = p.rs;

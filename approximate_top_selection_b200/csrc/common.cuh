@@ -51,6 +51,13 @@ __device__ __forceinline__ float fmin_nan(float a, float b) {
   return d;
 }
 
+// max that returns NaN when either operand is NaN (PTX max.NaN).
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // Programmatic dependent launch.  Kernels are launched so that they may start
 // while the previous kernel of the stream finishes; every thread waits here
 // (until that kernel has completed and its writes are visible) before it

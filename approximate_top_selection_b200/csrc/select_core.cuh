@@ -36,6 +36,10 @@ namespace tk {
 // NQ queues per thread: four for the float4 layout (k_b <= 2), one or two for
 // the wide k_b > 2 kernel.  The four-queue members (offer4, offer_tile, ...)
 // exist only for NQ == 4.
+#ifndef TOPK_MINMAX_QUEUES
+#define TOPK_MINMAX_QUEUES 1
+#endif
+
 template <int KB, int NQ = 4>
 struct Queues {
   float val[NQ][KB];
@@ -78,7 +82,33 @@ struct Queues {
     bool above[KB];
 #pragma unroll
     for (int s = 0; s < KB; ++s) above[s] = x > val[V][s];
+#if TOPK_MINMAX_QUEUES
+    if constexpr (KB <= 2) {
+    // The values as a max/min insertion network: slot s keeps the larger of
+    // itself and what the slots above pass down, and passes the smaller on.
+    // A NaN slot (only ever at the top) stays (max.NaN) and passes x on
+    // (fminf returns the non-NaN operand); with no NaN and x not -inf this
+    // is the sorted insert.  Each value depends on its own slot through one
+    // operation only, which shortens the chain between consecutive elements.
+    // Indices follow the strict comparisons, so ties keep the earlier element.
+    // Used for k_b <= 2 (the branch-free update of every element).
+#pragma unroll
+    for (int s = KB - 1; s > 0; --s)
+      idx[V][s] = above[s - 1] ? idx[V][s - 1] : (above[s] ? base : idx[V][s]);
+    idx[V][0] = above[0] ? base : idx[V][0];
+    float carry = x;
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      const float v = val[V][s];
+      val[V][s] = fmax_nan(v, carry);
+      if (s + 1 < KB) carry = fminf(v, carry);
+    }
+    } else {
+      place<V>(above, x, base);  // longer queues: the select chain measured faster
+    }
+#else
     place<V>(above, x, base);
+#endif
   }
 
   // Any x (NaN ranks above +inf; all NaNs tie).

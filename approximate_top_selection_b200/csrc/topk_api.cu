@@ -98,6 +98,7 @@ struct Plan {
   size_t ws_tickets = 0;  // bytes
   size_t ws_slots = 0;    // bytes
   int wide_nq = 0;        // k_b > 2 fast path: queues per thread of the 16-warp kernel
+  int layout = kLayoutSeparate;  // shared-memory layout of the streaming kernel (SelectLayout)
   size_t workspace() const { return ws_tickets + ws_slots; }
 };
 
@@ -200,34 +201,63 @@ int choose_grid(int64_t rows, int64_t E, int align, int64_t min_piece, int sms, 
 #define TOPK_WIDE_SPARSE 1
 #endif
 
+#ifndef TOPK_ALIAS_RING
+#define TOPK_ALIAS_RING 1
+#endif
+
+// Ring stages, shared memory and resident CTAs of a fast-path plan with the
+// given shared-memory layout (SelectLayout).
+template <typename KernelT>
+int fit_fast(KernelT kernel, int threads, int KB, int nl, int layout, Plan* pl,
+             const DeviceInfo& dev, int* per_sm) {
+  SelectSmem L{0, KB, pl->cand_cap, nl, layout};
+  pl->stages = fit_stages(L, 2);
+  L.stages = pl->stages;
+  pl->smem = L.total();
+  pl->layout = layout;
+  if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+  return occupancy(kernel, threads, pl->smem, per_sm);
+}
+
 template <typename T, int KB>
 int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& dev, Plan* pl) {
   const int C = b * KB;
   pl->cand_cap = sort_capacity(C);
   pl->align = fast ? Elem<T>::kAlign : 1;
   pl->wide_nq = 0;
+  pl->layout = kLayoutSeparate;
   int per_sm = 0;
-  if (fast && KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers) {
+  const int64_t E = rows * n;
+  if (fast) {
     // k_b > 2 with b >= 512: the 16-warp kernel, one lane per bucket (b lanes).
     // Smaller b keeps the 8-warp kernel, whose 256 lanes split a bucket over
     // fewer queues (fewer inserts).
-    pl->wide_nq = b > kWideConsumers ? b / kWideConsumers : 1;
-    const int nl = kWideConsumers * pl->wide_nq;
-    pl->stages = fit_stages(SelectSmem{0, KB, pl->cand_cap, nl}, 2);
-    SelectSmem L{pl->stages, KB, pl->cand_cap, nl};
-    pl->smem = L.total();
-    if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
-    int rc = pl->wide_nq == 1
-                 ? occupancy(bucket_select_wide<T, (KB > 2 ? KB : 3), 1>, kWideThreads, pl->smem, &per_sm)
-                 : occupancy(bucket_select_wide<T, (KB > 2 ? KB : 3), 2>, kWideThreads, pl->smem, &per_sm);
+    const bool wide = KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers;
+    pl->wide_nq = wide ? (b > kWideConsumers ? b / kWideConsumers : 1) : 0;
+    const int nl = wide ? kWideConsumers * pl->wide_nq : select_lanes(KB, b);
+    auto fit = [&](int layout) -> int {
+      if (!wide)
+        return fit_fast(bucket_select_tma<T, KB>, kPipeThreads, KB, nl, layout, pl, dev, &per_sm);
+      if (pl->wide_nq == 1)
+        return fit_fast(bucket_select_wide<T, (KB > 2 ? KB : 3), 1>, kWideThreads, KB, nl, layout,
+                        pl, dev, &per_sm);
+      return fit_fast(bucket_select_wide<T, (KB > 2 ? KB : 3), 2>, kWideThreads, KB, nl, layout, pl,
+                      dev, &per_sm);
+    };
+    int rc = fit(kLayoutSeparate);
     if (rc) return rc;
-  } else if (fast) {
-    pl->stages = fit_stages(SelectSmem{0, KB, pl->cand_cap, select_lanes(KB, b)}, 2);
-    SelectSmem L{pl->stages, KB, pl->cand_cap, select_lanes(KB, b)};
-    pl->smem = L.total();
-    if (pl->smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
-    int rc = occupancy(bucket_select_tma<T, KB>, kPipeThreads, pl->smem, &per_sm);
-    if (rc) return rc;
+    // One whole row per CTA (n a multiple of the alignment): every CTA streams
+    // a single piece, so its lane and Stage-2 buffers can share the ring.
+    if (TOPK_ALIAS_RING && n % pl->align == 0 &&
+        choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm) == rows) {
+      Plan keep = *pl;
+      const int keep_per_sm = per_sm;
+      rc = fit(kLayoutAliased);
+      if (rc || choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm) != rows) {
+        *pl = keep;  // not one row per CTA with the aliased layout: keep the plain one
+        per_sm = keep_per_sm;
+      }
+    }
   } else {
     pl->stages = 0;
     SelectSmem L{0, KB, pl->cand_cap, kLanes};
@@ -236,7 +266,6 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
     int rc = occupancy(bucket_select_general<T, KB>, kThreads, pl->smem, &per_sm);
     if (rc) return rc;
   }
-  const int64_t E = rows * n;
   pl->G = choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm);
   pl->units = E / pl->align;
   pl->ws_tickets = align_up(static_cast<size_t>(rows) * 4, 256);
@@ -365,14 +394,14 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 
 template <typename T, int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
+  const bool sample = a.tail.token != nullptr;
   if constexpr (KB > 2) {
     if (fast && pl.wide_nq > 0) {
-      const bool sample = a.tail.token != nullptr;
       auto go = [&](auto kernel) -> int {
         int rc = prepare_kernel(kernel);
         if (rc) return rc;
         return launch_pdl(kernel, dim3(pl.G), dim3(kWideThreads), pl.smem, st, a, pl.stages,
-                          pl.cand_cap);
+                          pl.cand_cap, pl.layout);
       };
       if (sample)
         return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1, true>)
@@ -380,15 +409,15 @@ int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStre
       return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1>) : go(bucket_select_wide<T, KB, 2>);
     }
   }
-  if (fast && a.tail.token != nullptr) {
+  if (fast && sample) {
     int rc = prepare_kernel(bucket_select_tma<T, KB, true>);
     if (rc) return rc;
     return launch_pdl(bucket_select_tma<T, KB, true>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st,
-                      a, pl.stages, pl.cand_cap);
+                      a, pl.stages, pl.cand_cap, pl.layout);
   }
   if (fast)
     return launch_pdl(bucket_select_tma<T, KB>, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a,
-                      pl.stages, pl.cand_cap);
+                      pl.stages, pl.cand_cap, pl.layout);
   return launch_pdl(bucket_select_general<T, KB>, dim3(pl.G), dim3(kThreads), pl.smem, st, a,
                     pl.cand_cap);
 }

@@ -778,6 +778,16 @@ def run_reference(args, world, rank, local):
                     "d2h_bytes_per_step": 0}}
 
 
+def _json_stdout():
+    """The one JSON line goes to the process's stdout; anything else a library
+    writes there (NCCL prints its version at start-up, for instance) is sent
+    to stderr instead, so that stdout holds exactly that line."""
+    out = os.fdopen(os.dup(1), "w")
+    sys.stdout.flush()
+    os.dup2(2, 1)
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -808,16 +818,17 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     if world != args.gpus:
         ap.error("--gpus %d but %d ranks were launched (WORLD_SIZE)" % (args.gpus, world))
+    out = _json_stdout()
     if args.impl == "reference":
         if rank != 0:
             return
         line = run_reference(args, world, rank, int(os.environ.get("LOCAL_RANK", "0")))
-        print(json.dumps(line))
+        print(json.dumps(line), file=out, flush=True)
         return
     world, rank, local = setup_dist(args)
     line = run_ours(args, world, rank, local)
     if rank == 0:
-        print(json.dumps(line))
+        print(json.dumps(line), file=out, flush=True)
     if torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
 

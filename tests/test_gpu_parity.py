@@ -420,3 +420,42 @@ def test_largest_candidate_sets_and_k(oracle_mod, b, kb, k):
         x = inputs.uniform_rows(rows, n, 4242 + b + kb + k + n)
         check_bucketed(x, k, b, kb, oracle_mod)
         _bf16_check(x.to(torch.bfloat16), k, b, kb, oracle_mod)
+
+
+# ------------------------------------------------------------------ one row per CTA
+@pytest.mark.parametrize("rows,n,k,b,kb", [(256, 65536, 50, 512, 1), (290, 32768, 512, 256, 2),
+                                           (200, 65536, 700, 1024, 4), (160, 40000, 64, 128, 3),
+                                           (148, 8192, 100, 64, 2)])
+def test_one_row_per_cta_layout(oracle_mod, rows, n, k, b, kb):
+    """A whole row per CTA: the queues' merge buffer and the Stage-2 buffer
+    share the tile ring.  Called through the binding and through the C ABI
+    with no workspace at all (none is needed), fp32 and bf16 rows, every
+    kernel (float4 queues, survivor queues, the 16-warp kernel)."""
+    lib = atk.load_library()
+    x = inputs.uniform_rows(rows, n, 5000 + rows + kb)
+    xd = x.to(DEV)
+    check_bucketed(x, k, b, kb, oracle_mod, x_dev=xd)
+    ov = torch.empty(rows, k, dtype=torch.float32, device=DEV)
+    oi = torch.empty(rows, k, dtype=torch.int32, device=DEV)
+    st = lib.topk_bucketed(xd.data_ptr(), rows, n, k, b, kb, ov.data_ptr(), oi.data_ptr(), None, 0,
+                           torch.cuda.current_stream().cuda_stream)
+    assert st == atk.TOPK_OK
+    torch.cuda.synchronize()
+    wv, wi = oracle_mod.bucketed(x.numpy(), k, b, kb)
+    assert np.array_equal(oi.cpu().numpy(), wi) and same_bits(ov.cpu().numpy(), wv)
+    _bf16_check(x.to(torch.bfloat16), k, b, kb, oracle_mod)
+
+
+@pytest.mark.parametrize("b,kb", [(512, 1), (256, 2), (512, 4)])
+def test_many_rows_sampling(oracle_mod, b, kb):
+    """The sampling draw on a row per CTA over more rows than SMs, fp32 and
+    bf16 logits."""
+    x = inputs.vocab_logits(256, 32768, 88 + kb)
+    u = torch.rand(256, generator=torch.Generator().manual_seed(9 + kb))
+    for dt in (torch.float32, torch.bfloat16):
+        xs = x.to(dt)
+        tok, v, i = atk.topk_sample(xs.to(DEV), 50, b, kb, 0.7, u.to(DEV))
+        ov, oi = oracle_mod.bucketed(xs.float().numpy(), 50, b, kb)
+        assert np.array_equal(i.cpu().numpy(), oi)
+        otok, margin = oracle_mod.sample_rows(ov, oi, 0.7, u.numpy().astype(np.float64))
+        assert np.all((tok.cpu().numpy() == otok) | (margin < 1e-5))
