@@ -96,6 +96,32 @@ struct SelectSmem {
   __host__ __device__ size_t total() const { return bar_off() + bar_bytes(); }
 };
 
+// Survivor masks on the FMA pipe (the k_b > 2 update saturates the ALU pipe):
+// FSET turns x > thr into 1.0 or 0.0 and an FMA adds it times 2^bit to 2^23,
+// exactly (the sum stays below 2^24), so the float's low mantissa bits are the
+// mask.  mask_acc_init / mask_acc_bits bracket the accumulation.
+__device__ __forceinline__ float mask_acc_init() { return 8388608.0f; }
+__device__ __forceinline__ float mask_acc_add(float acc, float x, float thr, int bit) {
+  return fmaf(x > thr ? 1.0f : 0.0f, static_cast<float>(1u << bit), acc);
+}
+__device__ __forceinline__ uint32_t mask_acc_bits(float acc) {
+  return __float_as_uint(acc) - 0x4B000000u;
+}
+
+// 0 * x is NaN exactly when x is NaN or infinite: false when any of the N
+// values is NaN or +-inf (FMA-pipe chains, two of them).
+template <int N>
+__device__ __forceinline__ bool all_finite(const float (&x)[N]) {
+  float a = 0.0f, b = 0.0f;
+#pragma unroll
+  for (int i = 0; i < N; i += 2) {
+    a = fmaf(x[i], 0.0f, a);
+    if (i + 1 < N) b = fmaf(x[i + 1], 0.0f, b);
+  }
+  const float s = a + b;
+  return s == s;
+}
+
 // k_b > 2: one tile (c valid floats at row positions pos_tile ...) for the
 // queues of this thread: element u sits at tile offset t + 256 u and feeds
 // queue u mod nq.  Each element is first compared with its queue's worst
@@ -115,8 +141,10 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
     x[u] = valid ? to_f32(tile[t + kThreads * u]) : __int_as_float(0x7f800000);
   }
   const uint32_t base = pos_tile + static_cast<uint32_t>(t);
-  if (!(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
-    // NaN or -inf somewhere in this thread's elements: exact update, in order.
+  const bool full = c >= static_cast<uint32_t>(kTile);
+  if (full ? !all_finite<U>(x) : !(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
+    // NaN or -inf (a full tile: or +inf) in this thread's elements: exact
+    // update, in order.
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (static_cast<uint32_t>(t + kThreads * u) >= c) continue;
@@ -132,7 +160,33 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
   // Survivor masks per queue (queue of element u is u mod nq; nq is 1, 2 or 4).
   uint32_t mask[4] = {0u, 0u, 0u, 0u};
   const float thr[4] = {q.val[0][KB - 1], q.val[1][KB - 1], q.val[2][KB - 1], q.val[3][KB - 1]};
-  if (nq == 1) {
+  if (full) {
+    // Every element valid: the masks on the FMA pipe, 16 bits per accumulator.
+    float lo[4], hi[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) lo[v] = hi[v] = mask_acc_init();
+    if (nq == 1) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (u < 16) lo[0] = mask_acc_add(lo[0], x[u], thr[0], u);
+        else hi[0] = mask_acc_add(hi[0], x[u], thr[0], u - 16);
+      }
+    } else if (nq == 2) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (u < 16) lo[u & 1] = mask_acc_add(lo[u & 1], x[u], thr[u & 1], u);
+        else hi[u & 1] = mask_acc_add(hi[u & 1], x[u], thr[u & 1], u - 16);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (u < 16) lo[u & 3] = mask_acc_add(lo[u & 3], x[u], thr[u & 3], u);
+        else hi[u & 3] = mask_acc_add(hi[u & 3], x[u], thr[u & 3], u - 16);
+      }
+    }
+#pragma unroll
+    for (int v = 0; v < 4; ++v) mask[v] = mask_acc_bits(lo[v]) | (mask_acc_bits(hi[v]) << 16);
+  } else if (nq == 1) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
       mask[0] |= (static_cast<uint32_t>(t + kThreads * u) < c && x[u] > thr[0]) ? (1u << u) : 0u;
@@ -178,10 +232,144 @@ __device__ __forceinline__ void select_tile_sparse(Queues<KB>& q, const T* tile,
 #undef TK_SURVIVORS
 }
 
+// ------------------------------------------------------------------ bf16 order keys
+// bfloat16 rows with k_b >= 2.  A bf16 value and its place in its queue fit in
+// one 32-bit word whose unsigned order is the method's total order: the high
+// half is a 16-bit order code of the value, the low half 0xFFFF minus the
+// element's ordinal in its queue (queues see their elements in increasing
+// position, so among equal values the earlier one compares larger).  A queue
+// is then KB such words, best first, and an element enters it through an
+// unsigned max/min insertion network -- 2 KB - 1 integer operations, no
+// comparison of indices and no branch, exact for every input.
+//
+// Order codes: a positive h codes as h ^ 0x8000 and a negative one as
+// (h ^ 0xFFFF) + 1, so that -0 and +0 share 0x8000, -inf codes 0x0080 and +inf
+// 0xFF80; every NaN codes 0xFFFF (all NaNs tie, above +inf).  No value codes 0,
+// so the word 0 marks an empty slot.  A queue's ordinal must fit 16 bits: the
+// path is taken for pieces of at most kKeyMaxPiece elements.
+constexpr int64_t kKeyMaxPiece = static_cast<int64_t>(kLanes) << 16;
+
+// Codes of the two bf16 in w (one per 16-bit half), w holding no NaN.  The
+// byte permute replicates each half's sign bit over that half (0xFFFF where
+// negative), so a negative half becomes (h ^ 0xFFFF) + 1 and a positive one
+// h ^ 0x8000; the +1 never carries across the halves.
+__device__ __forceinline__ uint32_t bf16x2_codes(uint32_t w) {
+  uint32_t m;  // selector nibbles 9 and B: bytes 1 and 3 with their sign bit replicated
+  asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(m) : "r"(w));
+  return (w ^ (m | 0x80008000u)) + (m & 0x00010001u);
+}
+
+// Codes of any two bf16 (NaN halves code 0xFFFF).
+__device__ __forceinline__ uint32_t bf16x2_codes_exact(uint32_t w) {
+  uint32_t c = bf16x2_codes(w);
+  if ((w & 0x7FFFu) > 0x7F80u) c |= 0x0000FFFFu;
+  if (((w >> 16) & 0x7FFFu) > 0x7F80u) c |= 0xFFFF0000u;
+  return c;
+}
+
+// acc + 0 * w on bf16 pairs (an FMA-pipe instruction): a half of the result is
+// NaN once any w offered to it held NaN or +-inf in that half.
+__device__ __forceinline__ uint32_t bf16x2_nonfinite_acc(uint32_t w, uint32_t acc) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(0u), "r"(acc));
+  return d;
+}
+
+__device__ __forceinline__ bool bf16x2_has_nan(uint32_t w) {
+  return ((w & 0x7FFFu) > 0x7F80u) | (((w >> 16) & 0x7FFFu) > 0x7F80u);
+}
+
+// Four queues per thread (the float4 layout: queue v of thread t takes the
+// positions congruent to 4t + v modulo kLanes), as order keys.  A key carries
+// its own tie-break, so the top-KB of a queue does not depend on the order in
+// which its elements are inserted: each queue is kept as SUB sub-queues that
+// take alternate stripes -- independent insertion chains, more work in flight
+// per thread -- and the sub-queues are combined when the piece ends.
+template <int KB, int SUB = 2>
+struct KeyQueues {
+  uint32_t key[4][SUB][KB];
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+#pragma unroll
+      for (int j = 0; j < SUB; ++j)
+#pragma unroll
+        for (int s = 0; s < KB; ++s) key[v][j][s] = 0u;
+  }
+
+  template <int V, int J>
+  __device__ __forceinline__ void insert(uint32_t x) {
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      const uint32_t k = key[V][J][s];
+      key[V][J][s] = max(k, x);
+      if (s + 1 < KB) x = min(k, x);
+    }
+  }
+
+  // Four consecutive bf16 (w.x: elements 0, 1; w.y: elements 2, 3), one per
+  // queue, at queue ordinal `ord`, into sub-queue J.
+  template <int J>
+  __device__ __forceinline__ void offer4(uint2 w, uint32_t ord, bool nan) {
+    const uint32_t lo = 0xFFFFu - ord;
+    const uint32_t cx = nan ? bf16x2_codes_exact(w.x) : bf16x2_codes(w.x);
+    const uint32_t cy = nan ? bf16x2_codes_exact(w.y) : bf16x2_codes(w.y);
+    // (low code << 16) | lo as cx * 2^16 + lo: a multiply-add, on the FMA pipe
+    // (the ALU pipe is the one the update saturates); the high code by a byte
+    // permute.
+    insert<0, J>(cx * 0x10000u + lo);
+    insert<1, J>(__byte_perm(cx, lo, 0x3254u));
+    insert<2, J>(cy * 0x10000u + lo);
+    insert<3, J>(__byte_perm(cy, lo, 0x3254u));
+  }
+
+  // Folds sub-queues 1.. into sub-queue 0.
+  __device__ __forceinline__ void combine() {
+#pragma unroll
+    for (int j = 1; j < SUB; ++j)
+#pragma unroll
+      for (int s = 0; s < KB; ++s) {
+        insert<0, 0>(key[0][j][s]);
+        insert<1, 0>(key[1][j][s]);
+        insert<2, 0>(key[2][j][s]);
+        insert<3, 0>(key[3][j][s]);
+      }
+  }
+
+  // Queue v (after combine()) as packed candidates at dst[0..KB); pos0 is the
+  // row position of its ordinal 0.
+  __device__ __forceinline__ void store(int v, uint64_t* dst, uint32_t pos0) const {
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      uint32_t k = 0u;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        if (w == v) k = key[w][0][s];
+      uint64_t out = 0ull;
+      if (k != 0u) {
+        const uint32_t code = k >> 16;
+        const uint32_t h = code >= 0x8000u ? (code ^ 0x8000u) : (((code - 1u) ^ 0xFFFFu) & 0xFFFFu);
+        const uint32_t ord = 0xFFFFu - (k & 0xFFFFu);
+        out = pack(order_key(__uint_as_float(h << 16)), pos0 + static_cast<uint32_t>(kLanes) * ord);
+      }
+      dst[s] = out;
+    }
+  }
+};
+
+#ifndef TOPK_BF16_KEYS
+#define TOPK_BF16_KEYS 1
+#endif
+#ifndef TOPK_BF16_KEYS_MIN_KB  // smallest k_b that takes the key path
+#define TOPK_BF16_KEYS_MIN_KB 2
+#endif
+
 // Register queues per CTA of the TMA kernel: four per thread (float4 layout)
-// for k_b <= 2, max(256, b) for the sparse k_b > 2 layout.
-__host__ __device__ __forceinline__ int select_lanes(int kb, int b) {
-  return kb <= 2 ? kLanes : (b > kThreads ? b : kThreads);
+// for k_b <= 2 and for the bf16 key path, max(256, b) for the sparse k_b > 2
+// layout.
+__host__ __device__ __forceinline__ int select_lanes(int kb, int b, bool keys = false) {
+  return kb <= 2 || keys ? kLanes : (b > kThreads ? b : kThreads);
 }
 
 constexpr int kConsumerWarps = kThreads / 32;
@@ -193,12 +381,14 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // the kThreads consumer threads never wait for each other inside a piece.
 // SAMPLE: the instantiation that also draws each row's token after Stage 2
 // (p.tail); without it the sampling code is not compiled in at all.
-template <typename T, int KB, bool SAMPLE = false>
+// KEYS: bf16 rows with k_b >= 2 in KeyQueues (see bf16 order keys).
+template <typename T, int KB, bool SAMPLE = false, bool KEYS = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
                                                                   int cand_cap, int layout) {
   constexpr int kTileElems = Elem<T>::kPerTile;
+  static_assert(!KEYS || sizeof(T) == 2, "the key path is for bf16 rows");
   extern __shared__ __align__(128) unsigned char smem[];
-  const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b), layout};
+  const SelectSmem L{stages, KB, cand_cap, select_lanes(KB, p.b, KEYS), layout};
   T* ring = reinterpret_cast<T*>(smem);
   uint64_t* lanebuf = reinterpret_cast<uint64_t*>(smem + L.lane_off());
   uint64_t* cand = reinterpret_cast<uint64_t*>(smem + L.cand_off());
@@ -267,9 +457,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
   // t + 256 q modulo nl = max(256, b) (select_tile_sparse), so each queue sees
   // four times more elements and only the survivors of a threshold test pay
   // for the sorted insert.
-  const int nl = select_lanes(KB, p.b);
+  const int nl = select_lanes(KB, p.b, KEYS);
   const int nq = nl / kThreads;
   Queues<KB> q;
+  KeyQueues<KB> kq;  // bf16 key path
   int st = 0;       // ring stage of the next tile
   uint32_t ph = 0;  // its full-barrier parity
   int64_t g = s0;
@@ -280,7 +471,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
     const uint32_t len = static_cast<uint32_t>(pend - g);  // < 2^31
     const uint32_t pos_thread = static_cast<uint32_t>(a) + 4u * tid;
-    q.reset();
+    if constexpr (KEYS)
+      kq.reset();
+    else
+      q.reset();
     for (uint32_t done = 0; done < len;) {
       const uint32_t c =
           (len - done) < static_cast<uint32_t>(kTileElems) ? (len - done) : kTileElems;
@@ -289,7 +483,44 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
                                  !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
         const T* stage_tile = ring + static_cast<size_t>(st) * kTileElems;
-        if (KB <= 2) {
+        if constexpr (KEYS) {
+          // In slices of kTile elements: stripe u of a slice is queue ordinal
+          // (done + hoff) / kLanes + u.  A pair NaN check per slice picks the
+          // cheap or the NaN-aware codes.
+          constexpr int U = kTile / kLanes;
+#pragma unroll
+          for (int h = 0; h < kTileElems / kTile; ++h) {
+            const uint32_t hoff = static_cast<uint32_t>(h * kTile);
+            const T* tile = stage_tile + hoff + 4 * tid;
+            const uint32_t ord0 = (done + hoff) / static_cast<uint32_t>(kLanes);
+            if (hoff + kTile <= c) {
+              uint2 w[U];
+#pragma unroll
+              for (int u = 0; u < U; ++u) w[u] = *reinterpret_cast<const uint2*>(tile + kLanes * u);
+              uint32_t mx = 0u, my = 0u;  // NaN or +-inf anywhere: the NaN-aware codes
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                mx = bf16x2_nonfinite_acc(w[u].x, mx);
+                my = bf16x2_nonfinite_acc(w[u].y, my);
+              }
+              const bool nan = bf16x2_has_nan(mx) | bf16x2_has_nan(my);
+#pragma unroll
+              for (int u = 0; u < U; u += 2) {
+                kq.template offer4<0>(w[u], ord0 + u, nan);
+                kq.template offer4<1>(w[u + 1], ord0 + u + 1, nan);
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                const uint32_t off = hoff + 4u * tid + static_cast<uint32_t>(kLanes * u);
+                if (off < c) {
+                  const uint2 w = *reinterpret_cast<const uint2*>(tile + kLanes * u);
+                  kq.template offer4<0>(w, ord0 + u, true);
+                }
+              }
+            }
+          }
+        } else if constexpr (KB <= 2) {
           // In slices of kTile elements (a bf16 tile holds two of them).
           constexpr int U = kTile / kLanes;
 #pragma unroll
@@ -345,7 +576,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
       group_sync(kThreads);
       if (*skip_flag) break;
     }
-    if (KB <= 2) {
+    if constexpr (KEYS) {
+      kq.combine();
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        kq.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB, pos_thread + v);
+    } else if constexpr (KB <= 2) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
     } else {
@@ -390,8 +626,10 @@ __device__ __forceinline__ void select_tile_wide(Queues<KB, NQ>& q, const T* til
     x[u] = valid ? to_f32(tile[t + CT * u]) : __int_as_float(0x7f800000);
   }
   const uint32_t base = pos_tile + static_cast<uint32_t>(t);
-  if (!(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
-    // NaN or -inf somewhere in this thread's elements: exact update, in order.
+  const bool full = c >= static_cast<uint32_t>(kTile);
+  if (full ? !all_finite<U>(x) : !(min_nan_all<U>(x) > __int_as_float(0xff800000))) {
+    // NaN or -inf (a full tile: or +inf) in this thread's elements: exact
+    // update, in order.
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (static_cast<uint32_t>(t + CT * u) >= c) continue;
@@ -410,10 +648,20 @@ __device__ __forceinline__ void select_tile_wide(Queues<KB, NQ>& q, const T* til
     mask[v] = 0u;
     thr[v] = q.val[v][KB - 1];
   }
+  if (full) {  // every element valid: the masks on the FMA pipe (U = 16 bits)
+    float acc[NQ];
 #pragma unroll
-  for (int u = 0; u < U; ++u)
-    mask[u % NQ] |=
-        (static_cast<uint32_t>(t + CT * u) < c && x[u] > thr[u % NQ]) ? (1u << u) : 0u;
+    for (int v = 0; v < NQ; ++v) acc[v] = mask_acc_init();
+#pragma unroll
+    for (int u = 0; u < U; ++u) acc[u % NQ] = mask_acc_add(acc[u % NQ], x[u], thr[u % NQ], u);
+#pragma unroll
+    for (int v = 0; v < NQ; ++v) mask[v] = mask_acc_bits(acc[v]);
+  } else {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      mask[u % NQ] |=
+          (static_cast<uint32_t>(t + CT * u) < c && x[u] > thr[u % NQ]) ? (1u << u) : 0u;
+  }
   // Survivors, software-pipelined as in select_tile_sparse.
   const T* tt = tile + t;
 #pragma unroll

@@ -99,6 +99,7 @@ struct Plan {
   size_t ws_slots = 0;    // bytes
   int wide_nq = 0;        // k_b > 2 fast path: queues per thread of the 16-warp kernel
   int layout = kLayoutSeparate;  // shared-memory layout of the streaming kernel (SelectLayout)
+  bool keys = false;      // bf16 rows with k_b >= 2 in order-key queues (KeyQueues)
   size_t workspace() const { return ws_tickets + ws_slots; }
 };
 
@@ -226,16 +227,27 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
   pl->align = fast ? Elem<T>::kAlign : 1;
   pl->wide_nq = 0;
   pl->layout = kLayoutSeparate;
+  pl->keys = false;
   int per_sm = 0;
   const int64_t E = rows * n;
   if (fast) {
-    // k_b > 2 with b >= 512: the 16-warp kernel, one lane per bucket (b lanes).
-    // Smaller b keeps the 8-warp kernel, whose 256 lanes split a bucket over
-    // fewer queues (fewer inserts).
-    const bool wide = KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers;
+    // bf16 rows with k_b >= 2 (rows short enough for 16-bit queue ordinals):
+    // order-key queues in the float4 layout.  Otherwise k_b > 2 with b >= 512:
+    // the 16-warp kernel, one lane per bucket (b lanes); smaller b keeps the
+    // 8-warp kernel, whose 256 lanes split a bucket over fewer queues (fewer
+    // inserts).
+    constexpr bool kKeyType = sizeof(T) == 2 && KB >= TOPK_BF16_KEYS_MIN_KB;
+    const bool keys = kKeyType && TOPK_BF16_KEYS && n <= kKeyMaxPiece;
+    pl->keys = keys;
+    const bool wide = !keys && KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers;
     pl->wide_nq = wide ? (b > kWideConsumers ? b / kWideConsumers : 1) : 0;
-    const int nl = wide ? kWideConsumers * pl->wide_nq : select_lanes(KB, b);
+    const int nl = wide ? kWideConsumers * pl->wide_nq : select_lanes(KB, b, keys);
     auto fit = [&](int layout) -> int {
+      if constexpr (kKeyType) {
+        if (keys)
+          return fit_fast(bucket_select_tma<T, KB, false, true>, kPipeThreads, KB, nl, layout, pl,
+                          dev, &per_sm);
+      }
       if (!wide)
         return fit_fast(bucket_select_tma<T, KB>, kPipeThreads, KB, nl, layout, pl, dev, &per_sm);
       if (pl->wide_nq == 1)
@@ -244,20 +256,18 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
       return fit_fast(bucket_select_wide<T, (KB > 2 ? KB : 3), 2>, kWideThreads, KB, nl, layout, pl,
                       dev, &per_sm);
     };
-    int rc = fit(kLayoutSeparate);
-    if (rc) return rc;
     // One whole row per CTA (n a multiple of the alignment): every CTA streams
-    // a single piece, so its lane and Stage-2 buffers can share the ring.
-    if (TOPK_ALIAS_RING && n % pl->align == 0 &&
-        choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm) == rows) {
-      Plan keep = *pl;
-      const int keep_per_sm = per_sm;
+    // a single piece, so its lane and Stage-2 buffers can share the ring.  The
+    // aliased layout is tried first (its smaller footprint can be what makes
+    // a row per CTA fit), the plain one otherwise.
+    int rc = TOPK_EUNSUPPORTED;
+    if (TOPK_ALIAS_RING && n % pl->align == 0) {
       rc = fit(kLayoutAliased);
-      if (rc || choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm) != rows) {
-        *pl = keep;  // not one row per CTA with the aliased layout: keep the plain one
-        per_sm = keep_per_sm;
-      }
+      if (!rc && choose_grid(rows, E, pl->align, kSelectMinPiece, dev.sms, per_sm) != rows)
+        rc = TOPK_EUNSUPPORTED;
     }
+    if (rc) rc = fit(kLayoutSeparate);
+    if (rc) return rc;
   } else {
     pl->stages = 0;
     SelectSmem L{0, KB, pl->cand_cap, kLanes};
@@ -407,6 +417,18 @@ int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStre
         return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1, true>)
                                : go(bucket_select_wide<T, KB, 2, true>);
       return pl.wide_nq == 1 ? go(bucket_select_wide<T, KB, 1>) : go(bucket_select_wide<T, KB, 2>);
+    }
+  }
+  if constexpr (sizeof(T) == 2 && KB >= TOPK_BF16_KEYS_MIN_KB) {
+    if (fast && pl.keys) {
+      auto go = [&](auto kernel) -> int {
+        int rc = prepare_kernel(kernel);
+        if (rc) return rc;
+        return launch_pdl(kernel, dim3(pl.G), dim3(kPipeThreads), pl.smem, st, a, pl.stages,
+                          pl.cand_cap, pl.layout);
+      };
+      return sample ? go(bucket_select_tma<T, KB, true, true>)
+                    : go(bucket_select_tma<T, KB, false, true>);
     }
   }
   if (fast && sample) {

@@ -273,8 +273,8 @@ def _kernel_name(cfg) -> str:
         return "score_select_umma" if _uses_tensor_cores(cfg) else "score_select_gemv"
     if cfg["kind"] == "rerank":
         return "rerank_kernel"
-    if cfg["kb"] > 2 and cfg["b"] >= 512:
-        return "bucket_select_wide"  # the 16-warp k_b > 2 kernel
+    if cfg["kb"] > 2 and cfg["b"] >= 512 and cfg.get("dtype") != "bf16":
+        return "bucket_select_wide"  # the 16-warp k_b > 2 kernel (bf16 rows: order-key queues)
     return "bucket_select_tma"
 
 

@@ -20,6 +20,7 @@ def test_kernel_choice_follows_the_library_dispatch():
     assert bench._kernel_name(bench.CONFIGS["vocab"]) == "bucket_select_tma"
     assert bench._kernel_name(bench.CONFIGS["long-b512-kb4"]) == "bucket_select_wide"
     assert bench._kernel_name(bench.CONFIGS["long-b256-kb4"]) == "bucket_select_tma"
+    assert bench._kernel_name(bench.CONFIGS["long-b512-kb4-bf16"]) == "bucket_select_tma"
     assert bench._kernel_name(bench.CONFIGS["decode-rerank"]) == "rerank_kernel"
 
 

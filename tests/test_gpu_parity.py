@@ -459,3 +459,28 @@ def test_many_rows_sampling(oracle_mod, b, kb):
         assert np.array_equal(i.cpu().numpy(), oi)
         otok, margin = oracle_mod.sample_rows(ov, oi, 0.7, u.numpy().astype(np.float64))
         assert np.all((tok.cpu().numpy() == otok) | (margin < 1e-5))
+
+
+# ------------------------------------------------------------------ bf16 order-key queues
+def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(bits.astype(np.uint16).view(np.int16)).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("kb", [2, 3, 4])
+def test_bf16_key_queues_special_bits(oracle_mod, kb):
+    """bf16 rows with k_b >= 2 run on 32-bit order keys (value code and queue
+    ordinal in one word).  Every special bit pattern must keep the total
+    order: NaNs of any sign and payload tie above +inf, -0 ties +0, -inf is
+    below every number, denormals order as numbers, equal values go by
+    index -- whole rows, split rows and ragged tails."""
+    rng = np.random.default_rng(700 + kb)
+    specials = np.array([0x7FC0, 0x7F81, 0xFFC1, 0x7FFF, 0xFF80, 0x7F80, 0x0000, 0x8000,
+                         0x0001, 0x8001, 0x007F, 0x807F, 0x3F80, 0xBF80], np.uint16)
+    for rows, n, k, b in [(6, 65536, 300, 256), (3, 400000, 700, 512), (40, 8200, 64, 1024),
+                          (2, 4104, 4096, 128)]:
+        bits = rng.integers(0x3E00, 0x4000, size=(rows, n)).astype(np.uint16)  # narrow: ties
+        bits[rng.random((rows, n)) < 0.3] |= 0x8000                          # negatives
+        pick = rng.random((rows, n)) < 0.02
+        bits[pick] = rng.choice(specials, size=int(pick.sum()))
+        x = _bf16_from_bits(bits)
+        _bf16_check(x, k, b, kb, oracle_mod)
