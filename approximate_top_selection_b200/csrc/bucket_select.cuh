@@ -365,11 +365,15 @@ struct KeyQueues {
 #define TOPK_BF16_KEYS_MIN_KB 2
 #endif
 
+#ifndef TOPK_SPARSE_MIN_KB  // smallest k_b that takes the survivor (sparse / wide) update
+#define TOPK_SPARSE_MIN_KB 3
+#endif
+
 // Register queues per CTA of the TMA kernel: four per thread (float4 layout)
-// for k_b <= 2 and for the bf16 key path, max(256, b) for the sparse k_b > 2
-// layout.
+// for the branch-free update (k_b < TOPK_SPARSE_MIN_KB) and for the bf16 key
+// path, max(256, b) for the sparse survivor layout.
 __host__ __device__ __forceinline__ int select_lanes(int kb, int b, bool keys = false) {
-  return kb <= 2 || keys ? kLanes : (b > kThreads ? b : kThreads);
+  return kb < TOPK_SPARSE_MIN_KB || keys ? kLanes : (b > kThreads ? b : kThreads);
 }
 
 constexpr int kConsumerWarps = kThreads / 32;
@@ -520,7 +524,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
               }
             }
           }
-        } else if constexpr (KB <= 2) {
+        } else if constexpr (KB < TOPK_SPARSE_MIN_KB) {
           // In slices of kTile elements (a bf16 tile holds two of them).
           constexpr int U = kTile / kLanes;
 #pragma unroll
@@ -581,7 +585,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
 #pragma unroll
       for (int v = 0; v < 4; ++v)
         kq.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB, pos_thread + v);
-    } else if constexpr (KB <= 2) {
+    } else if constexpr (KB < TOPK_SPARSE_MIN_KB) {
 #pragma unroll
       for (int v = 0; v < 4; ++v) q.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB);
     } else {

@@ -239,7 +239,7 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
     constexpr bool kKeyType = sizeof(T) == 2 && KB >= TOPK_BF16_KEYS_MIN_KB;
     const bool keys = kKeyType && TOPK_BF16_KEYS && n <= kKeyMaxPiece;
     pl->keys = keys;
-    const bool wide = !keys && KB > 2 && TOPK_WIDE_SPARSE && b >= kWideConsumers;
+    const bool wide = !keys && KB >= TOPK_SPARSE_MIN_KB && TOPK_WIDE_SPARSE && b >= kWideConsumers;
     pl->wide_nq = wide ? (b > kWideConsumers ? b / kWideConsumers : 1) : 0;
     const int nl = wide ? kWideConsumers * pl->wide_nq : select_lanes(KB, b, keys);
     auto fit = [&](int layout) -> int {
@@ -251,9 +251,9 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
       if (!wide)
         return fit_fast(bucket_select_tma<T, KB>, kPipeThreads, KB, nl, layout, pl, dev, &per_sm);
       if (pl->wide_nq == 1)
-        return fit_fast(bucket_select_wide<T, (KB > 2 ? KB : 3), 1>, kWideThreads, KB, nl, layout,
+        return fit_fast(bucket_select_wide<T, (KB >= TOPK_SPARSE_MIN_KB ? KB : 3), 1>, kWideThreads, KB, nl, layout,
                         pl, dev, &per_sm);
-      return fit_fast(bucket_select_wide<T, (KB > 2 ? KB : 3), 2>, kWideThreads, KB, nl, layout, pl,
+      return fit_fast(bucket_select_wide<T, (KB >= TOPK_SPARSE_MIN_KB ? KB : 3), 2>, kWideThreads, KB, nl, layout, pl,
                       dev, &per_sm);
     };
     // One whole row per CTA (n a multiple of the alignment): every CTA streams
@@ -405,7 +405,7 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
 template <typename T, int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
   const bool sample = a.tail.token != nullptr;
-  if constexpr (KB > 2) {
+  if constexpr (KB >= TOPK_SPARSE_MIN_KB) {
     if (fast && pl.wide_nq > 0) {
       auto go = [&](auto kernel) -> int {
         int rc = prepare_kernel(kernel);
