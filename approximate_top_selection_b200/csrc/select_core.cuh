@@ -273,21 +273,31 @@ __device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > 
 __device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a > b ? b : a; }
 
 // One compare-exchange round of the network (SIZE, STRIDE fixed at compile time).
+// Rounds whose stride crosses warps exchange through shared memory: with one
+// buffer (xchg2 == nullptr) each such round needs a barrier after its writes
+// and another after its reads (the next round rewrites the buffer); with two
+// buffers used in turn, the barrier after the next round's writes already
+// orders this round's reads before any rewrite, so one barrier per round.
 template <int EPT, int SIZE, int STRIDE>
-__device__ __forceinline__ void bitonic_round(uint64_t (&v)[EPT], uint64_t* xchg) {
+__device__ __forceinline__ void bitonic_round(uint64_t (&v)[EPT], uint64_t* xchg, uint64_t* xchg2,
+                                              int& flip) {
   const int t = threadIdx.x;
   if constexpr (STRIDE >= 32 * EPT) {
+    uint64_t* xb = (xchg2 != nullptr && flip) ? xchg2 : xchg;
 #pragma unroll
-    for (int j = 0; j < EPT; ++j) xchg[t * EPT + j] = v[j];
+    for (int j = 0; j < EPT; ++j) xb[t * EPT + j] = v[j];
     group_sync(kThreads);
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
       const int e = t * EPT + j;
-      const uint64_t o = xchg[e ^ STRIDE];
+      const uint64_t o = xb[e ^ STRIDE];
       const bool keep_max = ((e & SIZE) == 0) == ((e & STRIDE) == 0);
       v[j] = keep_max ? umax64(v[j], o) : umin64(v[j], o);
     }
-    group_sync(kThreads);
+    if (xchg2 == nullptr)
+      group_sync(kThreads);
+    else
+      flip ^= 1;
   } else if constexpr (STRIDE >= EPT) {
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
@@ -309,18 +319,23 @@ __device__ __forceinline__ void bitonic_round(uint64_t (&v)[EPT], uint64_t* xchg
       }
     }
   }
-  if constexpr (STRIDE > 1) bitonic_round<EPT, SIZE, STRIDE / 2>(v, xchg);
+  if constexpr (STRIDE > 1) bitonic_round<EPT, SIZE, STRIDE / 2>(v, xchg, xchg2, flip);
 }
 
 template <int EPT, int SIZE>
-__device__ __forceinline__ void bitonic_sizes(uint64_t (&v)[EPT], uint64_t* xchg) {
-  bitonic_round<EPT, SIZE, SIZE / 2>(v, xchg);
-  if constexpr (SIZE < kThreads * EPT) bitonic_sizes<EPT, SIZE * 2>(v, xchg);
+__device__ __forceinline__ void bitonic_sizes(uint64_t (&v)[EPT], uint64_t* xchg, uint64_t* xchg2,
+                                              int& flip) {
+  bitonic_round<EPT, SIZE, SIZE / 2>(v, xchg, xchg2, flip);
+  if constexpr (SIZE < kThreads * EPT) bitonic_sizes<EPT, SIZE * 2>(v, xchg, xchg2, flip);
 }
 
+// xchg2: nullable second exchange buffer of kThreads * EPT entries.
 template <int EPT>
-__device__ __forceinline__ void block_sort_desc(uint64_t (&v)[EPT], uint64_t* xchg) {
-  bitonic_sizes<EPT, 2>(v, xchg);
+__device__ __forceinline__ void block_sort_desc(uint64_t (&v)[EPT], uint64_t* xchg,
+                                                uint64_t* xchg2 = nullptr) {
+  int flip = 0;
+  bitonic_sizes<EPT, 2>(v, xchg, xchg2, flip);
+  if (xchg2 != nullptr) group_sync(kThreads);  // the last round's reads, before any reuse
 }
 
 // Bitonic network on the 32 * EPT keys of one warp, strided (lane l holds
@@ -383,7 +398,7 @@ __device__ __forceinline__ V negative_infinity() {
 
 template <int EPT, int VS, typename V>
 __device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                               int32_t* oi) {
+                                               int32_t* oi, uint64_t* xchg2) {
   constexpr int N = kThreads * EPT;
   const int t = threadIdx.x;
   uint64_t v[EPT];
@@ -393,7 +408,7 @@ __device__ __noinline__ void finalize_row_regs(uint64_t* cand, int C, int k, con
     v[j] = e < C ? cand[e] : 0ull;
   }
   group_sync(kThreads);  // cand is reused as the exchange buffer
-  block_sort_desc<EPT>(v, cand);
+  block_sort_desc<EPT>(v, cand, xchg2);
 #pragma unroll
   for (int j = 0; j < EPT; ++j) {
     const int e = t * EPT + j;
@@ -430,7 +445,8 @@ __host__ __device__ __forceinline__ size_t stage2_bytes(int C) {
 
 template <ValueSource VS, typename V>
 __device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                                  int32_t* oi);
+                                                  int32_t* oi, uint64_t* xchg2 = nullptr,
+                                                  int xchg2_cap = 0);
 
 // Stage 2 for a small k (k <= M = 32 * EPT, C <= 8 M): every warp sorts its M
 // candidates in registers, then in three rounds warp w < h takes the list of
@@ -494,7 +510,7 @@ __device__ __noinline__ void finalize_row_topk_warps(uint64_t* cand, int C, int 
 // and sort only those.  Same result as sorting all C and keeping k.
 template <int EPT, int VS, typename V>
 __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                                 int32_t* oi) {
+                                                 int32_t* oi, uint64_t* xchg2, int xchg2_cap) {
   const int t = threadIdx.x;
   uint32_t* hist = reinterpret_cast<uint32_t*>(cand + sort_capacity(C));  // 256 bins
   int* misc = reinterpret_cast<int*>(hist + 256);                        // digit, above, count, n
@@ -625,7 +641,7 @@ __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, c
   group_sync(kThreads);
   const int kept = misc[3];
   group_sync(kThreads);
-  finalize_row_fast<static_cast<ValueSource>(VS), V>(cand, kept, k, xrow, ov, oi);
+  finalize_row_fast<static_cast<ValueSource>(VS), V>(cand, kept, k, xrow, ov, oi, xchg2, xchg2_cap);
 }
 
 template <ValueSource VS, typename V>
@@ -634,20 +650,22 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
 
 template <int EPT, int VS, typename V>
 __device__ __noinline__ void finalize_row_select(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                                 int32_t* oi);
+                                                 int32_t* oi, uint64_t* xchg2, int xchg2_cap);
 
 // Stage 2 for the streaming kernels (kThreads threads): up to 8 keys per
 // thread are sorted in registers; larger candidate sets use the shared-memory
-// network.
+// network.  xchg2 (nullable, xchg2_cap entries): spare shared memory for a
+// second exchange buffer of the register sort.
 template <ValueSource VS, typename V>
 __device__ __forceinline__ void finalize_row_fast(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                                  int32_t* oi) {
+                                                  int32_t* oi, uint64_t* xchg2, int xchg2_cap) {
   const int ept = sort_capacity(C) / kThreads;
+  uint64_t* x2 = ept * kThreads <= xchg2_cap ? xchg2 : nullptr;
   switch (ept) {
-    case 1: finalize_row_regs<1, VS, V>(cand, C, k, xrow, ov, oi); break;
-    case 2: finalize_row_regs<2, VS, V>(cand, C, k, xrow, ov, oi); break;
-    case 4: finalize_row_regs<4, VS, V>(cand, C, k, xrow, ov, oi); break;
-    case 8: finalize_row_regs<8, VS, V>(cand, C, k, xrow, ov, oi); break;
+    case 1: finalize_row_regs<1, VS, V>(cand, C, k, xrow, ov, oi, x2); break;
+    case 2: finalize_row_regs<2, VS, V>(cand, C, k, xrow, ov, oi, x2); break;
+    case 4: finalize_row_regs<4, VS, V>(cand, C, k, xrow, ov, oi, x2); break;
+    case 8: finalize_row_regs<8, VS, V>(cand, C, k, xrow, ov, oi, x2); break;
     default: finalize_row<VS, V>(cand, C, k, xrow, ov, oi, kThreads); break;
   }
 }
@@ -682,9 +700,11 @@ __device__ __forceinline__ void finalize_row(uint64_t* cand, int C, int k, const
 #ifndef TOPK_WARP_TOPK
 #define TOPK_WARP_TOPK 1
 #endif
+// xchg2 (nullable, xchg2_cap entries): shared memory the caller no longer
+// needs, used as a second exchange buffer by the register sort.
 template <ValueSource VS, typename V>
 __device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xrow, V* ov,
-                                       int32_t* oi) {
+                                       int32_t* oi, uint64_t* xchg2 = nullptr, int xchg2_cap = 0) {
   if (TOPK_WARP_TOPK && C > k && C <= 8 * kThreads) {
     const int ept = sort_capacity(C) / kThreads;
     if (k <= 32 * ept) {
@@ -698,12 +718,12 @@ __device__ __forceinline__ void stage2(uint64_t* cand, int C, int k, const V* xr
   }
   if (C >= 1024 && 2 * k <= C && C <= 16 * kThreads) {
     switch (sort_capacity(C) / kThreads) {
-      case 4: finalize_row_select<4, VS, V>(cand, C, k, xrow, ov, oi); return;
-      case 8: finalize_row_select<8, VS, V>(cand, C, k, xrow, ov, oi); return;
-      default: finalize_row_select<16, VS, V>(cand, C, k, xrow, ov, oi); return;
+      case 4: finalize_row_select<4, VS, V>(cand, C, k, xrow, ov, oi, xchg2, xchg2_cap); return;
+      case 8: finalize_row_select<8, VS, V>(cand, C, k, xrow, ov, oi, xchg2, xchg2_cap); return;
+      default: finalize_row_select<16, VS, V>(cand, C, k, xrow, ov, oi, xchg2, xchg2_cap); return;
     }
   }
-  finalize_row_fast<VS, V>(cand, C, k, xrow, ov, oi);
+  finalize_row_fast<VS, V>(cand, C, k, xrow, ov, oi, xchg2, xchg2_cap);
 }
 
 // ------------------------------------------------------------------ sampling tail
@@ -814,10 +834,13 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
   const int C = b * KB;
   V* ov = out_vals + r * static_cast<int64_t>(k);
   int32_t* oi = out_idx + r * static_cast<int64_t>(k);
+  // After the lanes are merged their buffer is free: Stage 2 may use it.
+  uint64_t* spare = const_cast<uint64_t*>(lanebuf);
+  const int spare_cap = nl * KB;
   if (a == 0 && len == rs.n) {
     merge_lanes<KB>(lanebuf, b, 0, cand, T, nl);
     group_sync(T);
-    stage2<VS, V>(cand, C, k, xrow, ov, oi);
+    stage2<VS, V>(cand, C, k, xrow, ov, oi, spare, spare_cap);
     run_sample_tail<V>(tail, r, k, ov, oi);
     return;
   }
@@ -857,7 +880,7 @@ __device__ void finish_piece(const RowSplit& rs, int b, int k, int64_t r, int64_
     for (int s = 0; s < KB; ++s) cand[static_cast<size_t>(j) * KB + s] = best[s];
   }
   group_sync(T);
-  stage2<VS, V>(cand, C, k, xrow, ov, oi);
+  stage2<VS, V>(cand, C, k, xrow, ov, oi, spare, spare_cap);
   run_sample_tail<V>(tail, r, k, ov, oi);
   if (threadIdx.x == 0) rs.tickets[r] = 0u;  // leave the workspace zeroed
 }

@@ -402,6 +402,32 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cud
   return launch_status();
 }
 
+// launch_pdl for a kernel launched in clusters of cluster_x CTAs (along x).
+template <typename... KArgs, typename... Args>
+int launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  clear_launch_error();
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return TOPK_ECUDA;
+  }
+  return launch_status();
+}
+
 template <typename T, int KB>
 int launch_select_kb(bool fast, const Plan& pl, const SelectArgs<T>& a, cudaStream_t st) {
   const bool sample = a.tail.token != nullptr;
@@ -544,6 +570,64 @@ int tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000* out) {
   return TOPK_OK;
 }
 
+// The CTA-pair selector (score_select_umma_pair) serves 256 or more queries.
+#ifndef TOPK_UMMA_PAIR
+#define TOPK_UMMA_PAIR 1
+#endif
+constexpr int64_t kUmmaPairMinRows = 2 * kUmmaM;
+
+// Clusters of two CTAs of the pair kernel that can be resident at once on the
+// current device (cached per device and kernel): the grid's number of pairs.
+// 0 when the kernel does not fit.
+struct PairSlots {
+  int dev;
+  const void* fn;
+  int pairs;
+};
+PairSlots g_pair_slots[kOccSlots];
+int g_pair_n = 0;
+std::mutex g_pair_mu;
+
+template <typename KernelT>
+int umma_pair_slots(KernelT kernel, int threads, size_t smem, const DeviceInfo& dev, int* pairs) {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return TOPK_ECUDA;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  {
+    std::lock_guard<std::mutex> lk(g_pair_mu);
+    for (int i = 0; i < g_pair_n; ++i)
+      if (g_pair_slots[i].dev == d && g_pair_slots[i].fn == fn) {
+        *pairs = g_pair_slots[i].pairs;
+        return TOPK_OK;
+      }
+  }
+  *pairs = 0;
+  if (smem <= static_cast<size_t>(dev.max_smem_optin)) {
+    int rc = prepare_kernel(kernel);
+    if (rc) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * dev.sms));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      clusters = 0;  // no pair form on this device: the single-CTA kernel serves
+    }
+    *pairs = clusters;
+  }
+  std::lock_guard<std::mutex> lk(g_pair_mu);
+  if (g_pair_n < kOccSlots) g_pair_slots[g_pair_n++] = PairSlots{d, fn, *pairs};
+  return TOPK_OK;
+}
+
 template <int KB, int D>
 int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n, int b, int k,
                    float* out_vals, int32_t* out_idx, float* out_scores, void* ws,
@@ -580,20 +664,35 @@ int launch_umma_kd(const uint16_t* q, int64_t rows, const uint16_t* K, int64_t n
   a.n = n;
   a.b = b;
   a.T = static_cast<int>(T);
-  a.mtiles = static_cast<int>((rows + kUmmaM - 1) / kUmmaM);
   a.groups = b / kUmmaGroup;
   a.tiles_per_unit = static_cast<int>((T + kUmmaTPerTile - 1) / kUmmaTPerTile);
-  a.units = a.mtiles * a.groups;
   a.out_scores = out_scores;
   a.cand = static_cast<uint64_t*>(ws);
-  const size_t smem = UmmaSmem<D>::total;
-  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
-  if ((rc = prepare_kernel(score_select_umma<KB, D>))) return rc;
   if ((rc = prepare_kernel(umma_finish<KB>))) return rc;
-  const int grid = std::min(a.units, dev.sms);
-  if ((rc = launch_pdl(score_select_umma<KB, D>, dim3(grid), dim3(umma_threads(KB)), smem, st, tmQ,
-                       tmK, a)))
+  int pairs = 0;
+  if (TOPK_UMMA_PAIR && rows >= kUmmaPairMinRows &&
+      (rc = umma_pair_slots(score_select_umma_pair<KB, D>, umma_threads(KB), UmmaPairSmem<D>::total,
+                            dev, &pairs)))
     return rc;
+  if (pairs > 0) {
+    // A pair of CTAs per 256-query tile (cta_group::2).
+    a.mtiles = static_cast<int>((rows + kUmmaPairM - 1) / kUmmaPairM);
+    a.units = a.mtiles * a.groups;
+    const int grid = 2 * std::min(a.units, pairs);
+    if ((rc = launch_pdl_cluster(score_select_umma_pair<KB, D>, dim3(grid), dim3(umma_threads(KB)),
+                                 UmmaPairSmem<D>::total, st, 2, tmQ, tmK, a)))
+      return rc;
+  } else {
+    a.mtiles = static_cast<int>((rows + kUmmaM - 1) / kUmmaM);
+    a.units = a.mtiles * a.groups;
+    const size_t smem = UmmaSmem<D>::total;
+    if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
+    if ((rc = prepare_kernel(score_select_umma<KB, D>))) return rc;
+    const int grid = std::min(a.units, dev.sms);
+    if ((rc = launch_pdl(score_select_umma<KB, D>, dim3(grid), dim3(umma_threads(KB)), smem, st,
+                         tmQ, tmK, a)))
+      return rc;
+  }
   const size_t fsmem = stage2_bytes(b * KB);
   return launch_pdl(umma_finish<KB>, dim3(static_cast<unsigned>(rows)), dim3(kThreads), fsmem, st,
                     a.cand, rows, b, k, out_vals, out_idx);

@@ -317,6 +317,17 @@ def test_link_umma_shapes(oracle_mod, d, kb):
         check_scores(Q.to(DEV), K.to(DEV), k, b, kb, oracle_mod)
 
 
+@pytest.mark.parametrize("d", [128, 256])
+@pytest.mark.parametrize("kb", [1, 2, 4])
+def test_link_umma_pair_shapes(oracle_mod, d, kb):
+    """256 queries or more: the CTA-pair selector (tcgen05 cta_group::2, one
+    256-query tile per pair).  Ragged query tiles (the second CTA's rows past
+    the end) and stripe counts that are not a multiple of the 32-stripe tile."""
+    for (rows, T, b, k) in [(256, 32, 64, 50), (300, 37, 64, 100), (600, 70, 256, 300)]:
+        Q, K = inputs.link_inputs(rows, T * b, d, 51 + rows + d + kb)
+        check_scores(Q.to(DEV), K.to(DEV), k, b, kb, oracle_mod)
+
+
 def test_link_umma_special_values(oracle_mod):
     """Scores that are +-inf or NaN (from inf / NaN inputs) take the exact
     queue update: the selection on the GPU's scores is still the oracle's."""
