@@ -270,7 +270,9 @@ def _uses_tensor_cores(cfg) -> bool:
 
 def _kernel_name(cfg) -> str:
     if cfg["kind"] == "score":
-        return "score_select_umma" if _uses_tensor_cores(cfg) else "score_select_gemv"
+        if _uses_tensor_cores(cfg):  # CTA pairs from 256 queries on
+            return "score_select_umma_pair" if cfg["queries"] >= 256 else "score_select_umma"
+        return "score_select_gemv"
     if cfg["kind"] == "rerank":
         return "rerank_kernel"
     if cfg["kb"] > 2 and cfg["b"] >= 512 and cfg.get("dtype") != "bf16":
@@ -603,6 +605,7 @@ _KERNEL_SOURCES = {
     "bucket_select_wide": ("common.cuh", "select_core.cuh", "bucket_select.cuh"),
     "score_select_gemv": ("common.cuh", "select_core.cuh", "score_gemv.cuh"),
     "score_select_umma": ("common.cuh", "select_core.cuh", "score_umma.cuh"),
+    "score_select_umma_pair": ("common.cuh", "select_core.cuh", "score_umma.cuh"),
     "rerank_kernel": ("common.cuh", "select_core.cuh", "rerank.cuh"),
 }
 

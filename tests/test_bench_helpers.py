@@ -16,7 +16,7 @@ def test_every_config_names_a_kernel_with_sources():
 
 def test_kernel_choice_follows_the_library_dispatch():
     assert bench._kernel_name(bench.CONFIGS["decode"]) == "score_select_gemv"
-    assert bench._kernel_name(bench.CONFIGS["link"]) == "score_select_umma"
+    assert bench._kernel_name(bench.CONFIGS["link"]) == "score_select_umma_pair"
     assert bench._kernel_name(bench.CONFIGS["vocab"]) == "bucket_select_tma"
     assert bench._kernel_name(bench.CONFIGS["long-b512-kb4"]) == "bucket_select_wide"
     assert bench._kernel_name(bench.CONFIGS["long-b256-kb4"]) == "bucket_select_tma"
