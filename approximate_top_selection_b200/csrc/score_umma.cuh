@@ -546,7 +546,7 @@ __global__ void __launch_bounds__(umma_threads(KB), 1)
 constexpr int kUmmaPairM = 2 * kUmmaM;                           // 256 queries per unit
 constexpr int kUmmaPairStageBytes = kUmmaStageBytes / 2;         // 128 key rows x 64 bf16
 #ifndef TOPK_UMMA_PAIR_STAGES
-#define TOPK_UMMA_PAIR_STAGES 8
+#define TOPK_UMMA_PAIR_STAGES 4
 #endif
 constexpr int kUmmaPairStages = TOPK_UMMA_PAIR_STAGES;
 // Accumulator buffers of 256 TMEM columns (2: the epilogue drains one while
