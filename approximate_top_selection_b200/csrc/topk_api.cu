@@ -910,10 +910,10 @@ int score_rerank(const uint16_t* q, int64_t rows, int d, const uint16_t* K, int6
   DeviceInfo dev;
   int rc = current_device_info(&dev);
   if (rc) return rc;
-  const size_t smem = stage2_bytes(c) + static_cast<size_t>(rerank_table_size(c)) * 4 + 16;
-  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
   RerankArgs a{q, K, cand_idx, rows, n, k_batch_stride, c, k, out_vals, out_idx, out_scores};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = stage2_bytes(c) + static_cast<size_t>(rerank_table_size(c)) * 4 + 16;
+  if (smem > static_cast<size_t>(dev.max_smem_optin)) return TOPK_EUNSUPPORTED;
   const dim3 grid(static_cast<unsigned>(rows)), block(kThreads);
   if (d == 128) {
     if ((rc = prepare_kernel(rerank_kernel<128>))) return rc;

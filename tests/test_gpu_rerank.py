@@ -101,6 +101,39 @@ def test_rerank_per_row_keys(oracle_mod, rows, n, d, c, k):
     assert atk.topk_device_status() == 0
 
 
+@pytest.mark.parametrize("rows,n,d,supports,size,k", [
+    (64, 32768, 128, 4, 512, 512),   # ~960 distinct of 2048 slots: the k best selected, then 512 sorted
+    (40, 32768, 256, 4, 512, 512),
+    (48, 8192, 128, 2, 256, 200),    # ~330 distinct: select 200, sort 256
+    (48, 8192, 128, 2, 256, 100),
+])
+def test_rerank_select_before_sort(oracle_mod, rows, n, d, supports, size, k):
+    """Distinct-candidate counts whose sort shrinks to the next smaller power
+    of two once only the k best are kept (the decode re-rank shape among them)."""
+    q = inputs.bf16_normal((rows, d), 1.0, 0xB6 + d, device=DEV)
+    K = inputs.bf16_normal((rows, n, d), d ** -0.5, 0xB7 + d, device=DEV)
+    cand = inputs.support_union(rows, n, supports, size, 0xB8 + k).numpy()
+    distinct = [len(set(r.tolist())) for r in cand]
+    assert min(distinct) > k and max(distinct) <= 2 * max(k, 256) - 1, distinct[:4]
+    check_rerank(q, K, cand, k, oracle_mod)
+    assert atk.topk_device_status() == 0
+
+
+@pytest.mark.parametrize("rows,n,d,c,k,shared", [
+    (700, 1000, 128, 2048, 512, False),   # more rows than 4 CTAs x 148 SMs: a second wave
+    (301, 100000, 256, 1000, 100, True),  # one key matrix for all rows; n > 32 * 2048: hash set
+    (400, 1000, 128, 300, 64, False),
+])
+def test_rerank_many_rows(oracle_mod, rows, n, d, c, k, shared):
+    """Hundreds of rows (one CTA each), per-row and shared key matrices, the
+    bitmap and the hash-set listing."""
+    q = inputs.bf16_normal((rows, d), 1.0, 0xB9 + d, device=DEV)
+    shape = (n, d) if shared else (rows, n, d)
+    K = inputs.bf16_normal(shape, d ** -0.5, 0xBA + d, device=DEV)
+    check_rerank(q, K, _supports(rows, n, c, rows + c), k, oracle_mod)
+    assert atk.topk_device_status() == 0
+
+
 def test_rerank_shared_keys(oracle_mod):
     rows, n, d, c, k = 64, 65536, 256, 1000, 100
     q = inputs.bf16_normal((rows, d), d ** -0.5, 0xB2, device=DEV)
