@@ -75,6 +75,30 @@ __device__ __forceinline__ float fmin3_nan(float a, float b, float c) {
   return d;
 }
 
+// Three-input max that keeps NaN (sm_100).
+__device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// NaN-keeping maximum of N values (three-input steps).
+template <int N>
+__device__ __forceinline__ float max_nan_all(const float (&v)[N]) {
+  float m[(N + 2) / 3];
+#pragma unroll
+  for (int i = 0; i < (N + 2) / 3; ++i) {
+    const float a = v[3 * i];
+    const float b = 3 * i + 1 < N ? v[3 * i + 1] : a;
+    const float c = 3 * i + 2 < N ? v[3 * i + 2] : a;
+    m[i] = fmax3_nan(a, b, c);
+  }
+  if constexpr ((N + 2) / 3 == 1)
+    return m[0];
+  else
+    return max_nan_all<(N + 2) / 3>(m);
+}
+
 // NaN-keeping minimum of N values (three-input steps).
 template <int N>
 __device__ __forceinline__ float min_nan_all(const float (&v)[N]) {

@@ -215,6 +215,10 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 // ------------------------------------------------------------------ queues
+#ifndef TOPK_UMMA_TILE_MAX  // k_b = 1: the maximum of each 32-score load first
+#define TOPK_UMMA_TILE_MAX 1
+#endif
+
 // NQ bucket queues of KB entries (value domain, as Queues in select_core.cuh),
 // storing true entity indices.
 template <int NQ, int KB>
@@ -278,7 +282,6 @@ __device__ __forceinline__ void umma_feed_bucket(BucketQueues<NQ, KB>& q, const 
   float all[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) all[i] = __uint_as_float(r[i]);
-  const bool special = !(min_nan_all<32>(all) > __int_as_float(0xff800000));
   const int valid = T - t0 < 32 ? T - t0 : 32;  // stripes of this tile inside the tensor
   if (out_scores != nullptr && row < rows) {
 #pragma unroll
@@ -286,6 +289,32 @@ __device__ __forceinline__ void umma_feed_bucket(BucketQueues<NQ, KB>& q, const 
       if (i < valid)
         out_scores[row * n + static_cast<int64_t>(t0 + i) * b + jb] = __uint_as_float(r[i]);
   }
+  if constexpr (KB == 1 && TOPK_UMMA_TILE_MAX) {
+    // One queue entry takes the best of the 32: the load's maximum (a NaN-
+    // keeping max tree, about one ALU instruction per two scores) replaces
+    // the queue's entry only if it is strictly larger, at its first position
+    // among the 32 (the lowest stripe: ties go to the lower index).  The
+    // element-wise path below takes loads whose maximum is NaN or -inf (NaN
+    // ranks above everything, -inf must still fill an empty queue) or zero
+    // (the element holding it may be -0 while the maximum reads +0); any
+    // other maximum has the bits of the elements equal to it.
+    const float m = max_nan_all<32>(all);
+    if (valid == 32 && m > __int_as_float(0xff800000) && m != 0.0f) {
+      if (m > q.val[QI][0]) {
+        uint32_t hit = 0u;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hit |= (all[i] == m ? 1u : 0u) << i;
+        q.val[QI][0] = m;
+        q.idx[QI][0] = static_cast<uint32_t>(t0 + __ffs(static_cast<int>(hit)) - 1);
+      }
+      return;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid) q.template insert_exact<QI>(__uint_as_float(r[i]), static_cast<uint32_t>(t0 + i));
+    return;
+  }
+  const bool special = !(min_nan_all<32>(all) > __int_as_float(0xff800000));
   if (!special && valid == 32) {
 #pragma unroll
     for (int i = 0; i < 32; ++i)
@@ -786,8 +815,12 @@ __global__ void __launch_bounds__(umma_threads(KB), 1)
 
 // Stage 2 of the tensor-core path: per query, the exact top-k of the b*k_b
 // bucket candidates (the workspace is cleared behind the reads).
+#ifndef TOPK_FINISH_MIN_CTAS  // resident CTAs per SM the register budget is cut for
+#define TOPK_FINISH_MIN_CTAS 6
+#endif
 template <int KB>
-__global__ void __launch_bounds__(kThreads) umma_finish(uint64_t* cand_ws, int64_t rows, int b,
+__global__ void __launch_bounds__(kThreads, TOPK_FINISH_MIN_CTAS)
+    umma_finish(uint64_t* cand_ws, int64_t rows, int b,
                                                         int k, float* out_vals, int32_t* out_idx) {
 
   extern __shared__ __align__(128) unsigned char smem[];

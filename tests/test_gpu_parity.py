@@ -340,6 +340,29 @@ def test_link_umma_special_values(oracle_mod):
     assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
 
 
+@pytest.mark.parametrize("rows", [64, 256])
+def test_link_umma_kb1_special_values(oracle_mod, rows):
+    """k_b = 1 takes each 32-score load's maximum before touching its queue:
+    ties inside one load and across loads of a bucket, zero maxima (a zero
+    query: every score is +0 or -0), +-inf and NaN scores must select exactly
+    as the oracle does on the GPU's own scores (64 rows: one CTA per tile, 256:
+    CTA pairs)."""
+    b = 64
+    Q, K = inputs.link_inputs(rows, 64 * b, 128, 43)   # 64 stripes per bucket: two loads each
+    Q[1:4] = Q[0]                    # four queries share the tied maxima below
+    Q[5] = 0.0                       # all scores +-0
+    top = Q[0].float() * 8.0
+    for key in (10, 10 + b, 10 + 2 * b, 20 + 3 * b, 20 + 40 * b):  # same load / across loads
+        K[key] = top.to(K.dtype)
+    K[7] = float("inf")
+    K[8 + 33 * b] = -float("inf")
+    K[9 + 5 * b, 3] = float("nan")
+    v, i, s = atk.score_topk(Q.to(DEV), K.to(DEV), 40, b, 1, return_scores=True)
+    ov, oi = oracle_mod.bucketed(s.cpu().numpy(), 40, b, 1)
+    assert np.array_equal(i.cpu().numpy(), oi) and same_bits(v.cpu().numpy(), ov)
+    assert atk.topk_device_status() == 0
+
+
 def test_link_config_full(oracle_mod):
     """1024 queries x 2^20 entities, d = 256, k = 100, b = 1024, k_b = 1:
     sampled query rows against the fp64 oracle."""
