@@ -486,17 +486,19 @@ def run_ours(args, world, rank, local):
         for i in range(args.warmup):
             run[i % nrot]()
     barrier(world)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     with ClockSampler(local) as clk:
         barrier(world)
-        ev0.record(stream)
+        evs[0].record(stream)
         for i in range(args.steps):
             run[i % nrot]()
-        ev1.record(stream)
+            evs[i + 1].record(stream)
         barrier(world)
-    ms = ev0.elapsed_time(ev1)
+    ms = evs[0].elapsed_time(evs[-1])
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
+    dist = step_distribution(evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps))
+    dist = {key: max_over_ranks(v, world) for key, v in dist.items()}
     hbm, tflops_burst, peak_src = _peaks()
     achieved = w.bytes / (ms_step * 1e-3) / 1e9
     line = {
@@ -507,6 +509,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
+        "step_ms": dist,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -553,6 +556,14 @@ def _graph_of_steps(works, reps: int):
     return g
 
 
+def step_distribution(per_step_ms) -> dict:
+    """Median and 90th percentile (nearest rank) of per-step times in ms."""
+    xs = sorted(float(x) for x in per_step_ms)
+    if not xs:
+        return {"median": None, "p90": None}
+    return {"median": statistics.median(xs), "p90": xs[max(0, math.ceil(0.9 * len(xs)) - 1)]}
+
+
 def sweep_cell(name: str, dev, local: int, min_region_s: float = 0.25) -> dict:
     """One workload timed alone: CUDA-graph replays of back-to-back steps over
     rotating input copies, CUDA events around the replays, clocks sampled
@@ -568,22 +579,24 @@ def sweep_cell(name: str, dev, local: int, min_region_s: float = 0.25) -> dict:
     est = _time_ms(g.replay, 3, warmup=0) / per_replay
     replays = max(3, math.ceil(min_region_s * 1e3 / (est * per_replay)))
     stream = torch.cuda.current_stream()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(replays + 1)]
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(replays):
+        evs[0].record(stream)
+        for i in range(replays):
             g.replay()
-        ev1.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize()
     steps = replays * per_replay
-    ms = ev0.elapsed_time(ev1) / steps
+    ms = evs[0].elapsed_time(evs[-1]) / steps
+    # per step, from each replay's own events (one replay = per_replay steps)
+    dist = step_distribution(evs[i].elapsed_time(evs[i + 1]) / per_replay for i in range(replays))
     hbm, _, peak_src = _peaks()
     gbs = w.bytes / (ms * 1e-3) / 1e9
     roof = _roofline(w, ms, gbs, hbm, peak_src, ms * steps * 1e-3)
     out = {"ms_per_step": ms, "GB/s": gbs, "rows_per_s": w.rows / (ms * 1e-3),
            "bound": roof["bound"], "achieved": roof["achieved"], "unit": roof["unit"],
-           "frac": roof["frac"], "kernel": roof["kernel"], "steps": steps,
+           "frac": roof["frac"], "kernel": roof["kernel"], "steps": steps, "step_ms": dist,
            "l2": _l2_note(w, nrot), "clocks": clk.summary()}
     del g, works, w
     torch.cuda.synchronize()

@@ -89,3 +89,13 @@ def test_split_workload_launches():
 
 def test_job_throughput_is_weak_scaling():
     assert math.isclose(bench.job_throughput(1e9, 2.0, 4), 4 * 1e9 / 2e-3 / 1e9)
+
+
+def test_step_distribution():
+    """Median and nearest-rank 90th percentile of the per-step times."""
+    d = bench.step_distribution([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert d == {"median": 3.0, "p90": 5.0}
+    d = bench.step_distribution([float(x) for x in range(1, 21)])  # 1..20
+    assert d["median"] == 10.5 and d["p90"] == 18.0
+    assert bench.step_distribution([7.0]) == {"median": 7.0, "p90": 7.0}
+    assert bench.step_distribution([]) == {"median": None, "p90": None}

@@ -14,7 +14,8 @@ pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
-        "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "gpu_launches", "clocks"}
+        "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "gpu_launches", "clocks",
+        "step_ms"}
 
 
 def _run(*args):
@@ -38,6 +39,8 @@ def test_bench_line(extra):
     e = d["e2e"]
     assert e["h2d_bytes_per_step"] == 8 * 4096 * 4 and e["d2h_bytes_per_step"] == 8 * 64 * 8
     assert d["gpu_launches"] == 20
+    st = d["step_ms"]
+    assert 0 < st["median"] <= st["p90"]
 
 
 def test_reference_line():
@@ -64,6 +67,7 @@ def test_default_line_carries_the_sweep():
     for name, cell in sw.items():
         assert cell["ms_per_step"] > 0 and 0 < cell["frac"] < 1.5, name
         assert cell["bound"] in ("hbm", "tensor"), name
+        assert 0 < cell["step_ms"]["median"] <= cell["step_ms"]["p90"], name
 
 
 def test_split_workload_one_gpu():
