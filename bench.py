@@ -394,17 +394,26 @@ def cpu_baseline(w: Workload, budget_s: float = 10.0):
         step()
         return time.perf_counter() - t0
 
-    probe = min(w.rows, max(1, threads))
-    t = run(probe)
-    rows = int(min(w.rows, max(probe, probe * budget_s / max(t, 1e-6))))
-    if rows > probe:
-        t = run(rows)
-    else:
-        rows = probe
+    def sample(nthreads, budget):
+        oracle.set_threads(nthreads)
+        probe = min(w.rows, max(1, nthreads))
+        t = run(probe)
+        rows = int(min(w.rows, max(probe, probe * budget / max(t, 1e-6))))
+        if rows > probe:
+            t = run(rows)
+        else:
+            rows = probe
+        return rows, t
+
     per_row = w.bytes / w.rows
+    rows1, t1 = sample(1, budget_s / 4)
+    rows, t = sample(threads, budget_s)
     return {"value": rows * per_row / t / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": "%d of %d rows of the %s workload (%.1f s)" % (rows, w.rows, w.name, t),
-            "rows_per_s": rows / t}
+            "rows_per_s": rows / t,
+            "single_thread": {"value": rows1 * per_row / t1 / 1e9, "unit": "GB/s",
+                              "rows_per_s": rows1 / t1,
+                              "sample": "%d of %d rows (%.1f s)" % (rows1, w.rows, t1)}}
 
 
 # ---------------------------------------------------------------- runs
