@@ -279,6 +279,72 @@ __device__ __forceinline__ bool bf16x2_has_nan(uint32_t w) {
   return ((w & 0x7FFFu) > 0x7F80u) | (((w >> 16) & 0x7FFFu) > 0x7F80u);
 }
 
+// k_b = 1 on bf16 rows: a thread's four queues (the float4 layout) as two
+// bf16x2 value words (queues 0, 1 and 2, 3) and two words of 16-bit stripe
+// ordinals (0xFFFF: empty), so that one packed compare and two bit-selects
+// update two queues.  A finite element replaces its queue's entry when it is
+// strictly larger (ties keep the earlier stripe; -0 and +0 compare equal);
+// the entry starts at -inf, which every finite element beats.  A slice that
+// holds a NaN or +-inf takes the element-wise update under the total order
+// (16-bit order codes: NaN above +inf, -0 = +0, an empty queue takes anything).
+__device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
+  uint32_t d;  // per half: 0xFFFF where a > b, else 0
+  asm("set.gt.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bf16_order_code(uint32_t h) {
+  if ((h & 0x7FFFu) > 0x7F80u) return 0xFFFFu;      // NaN
+  return (h & 0x8000u) ? ((h ^ 0xFFFFu) + 1u) & 0xFFFFu : (h ^ 0x8000u);
+}
+
+struct PairQueues {
+  uint32_t val[2], ord[2];
+
+  __device__ __forceinline__ void reset() {
+    val[0] = val[1] = 0xFF80FF80u;  // -inf, -inf
+    ord[0] = ord[1] = 0xFFFFFFFFu;  // empty, empty
+  }
+
+  // Four consecutive finite bf16 (w.x: queues 0, 1; w.y: queues 2, 3) at
+  // stripe ordinal o.
+  __device__ __forceinline__ void offer4(uint2 w, uint32_t o) {
+    const uint32_t o2 = o * 0x00010001u;
+    const uint32_t m0 = bf16x2_gt_mask(w.x, val[0]);
+    const uint32_t m1 = bf16x2_gt_mask(w.y, val[1]);
+    val[0] = (w.x & m0) | (val[0] & ~m0);
+    ord[0] = (o2 & m0) | (ord[0] & ~m0);
+    val[1] = (w.y & m1) | (val[1] & ~m1);
+    ord[1] = (o2 & m1) | (ord[1] & ~m1);
+  }
+
+  __device__ __forceinline__ void offer4_exact(uint2 w, uint32_t o) {
+    const uint32_t in[2] = {w.x, w.y};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int word = e >> 1, sh = (e & 1) * 16;
+      const uint32_t h = (in[word] >> sh) & 0xFFFFu;
+      const uint32_t cur = (val[word] >> sh) & 0xFFFFu;
+      const uint32_t co = (ord[word] >> sh) & 0xFFFFu;
+      if (co == 0xFFFFu || bf16_order_code(h) > bf16_order_code(cur)) {
+        val[word] = (val[word] & ~(0xFFFFu << sh)) | (h << sh);
+        ord[word] = (ord[word] & ~(0xFFFFu << sh)) | (o << sh);
+      }
+    }
+  }
+
+  // Queue v as one packed (order key, ~position) word, position = pos_thread
+  // + v + ordinal * kLanes (0: empty).
+  __device__ __forceinline__ void store(int v, uint64_t* dst, uint32_t pos_thread) const {
+    const int word = v >> 1, sh = (v & 1) * 16;
+    const uint32_t o = (ord[word] >> sh) & 0xFFFFu;
+    const uint32_t h = (val[word] >> sh) & 0xFFFFu;
+    dst[0] = o == 0xFFFFu ? 0ull
+                          : pack(order_key(__uint_as_float(h << 16)),
+                                 pos_thread + static_cast<uint32_t>(v) + o * static_cast<uint32_t>(kLanes));
+  }
+};
+
 // Four queues per thread (the float4 layout: queue v of thread t takes the
 // positions congruent to 4t + v modulo kLanes), as order keys.  A key carries
 // its own tie-break, so the top-KB of a queue does not depend on the order in
@@ -361,8 +427,8 @@ struct KeyQueues {
 #ifndef TOPK_BF16_KEYS
 #define TOPK_BF16_KEYS 1
 #endif
-#ifndef TOPK_BF16_KEYS_MIN_KB  // smallest k_b that takes the key path
-#define TOPK_BF16_KEYS_MIN_KB 2
+#ifndef TOPK_BF16_KEYS_MIN_KB  // smallest k_b that takes the key path (k_b = 1: PairQueues)
+#define TOPK_BF16_KEYS_MIN_KB 1
 #endif
 
 #ifndef TOPK_SPARSE_MIN_KB  // smallest k_b that takes the survivor (sparse / wide) update
@@ -385,7 +451,8 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // the kThreads consumer threads never wait for each other inside a piece.
 // SAMPLE: the instantiation that also draws each row's token after Stage 2
 // (p.tail); without it the sampling code is not compiled in at all.
-// KEYS: bf16 rows with k_b >= 2 in KeyQueues (see bf16 order keys).
+// KEYS: bf16 rows on 16-bit codes -- k_b >= 2 in KeyQueues (see bf16 order
+// keys), k_b = 1 in PairQueues.
 template <typename T, int KB, bool SAMPLE = false, bool KEYS = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
                                                                   int cand_cap, int layout) {
@@ -464,7 +531,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
   const int nl = select_lanes(KB, p.b, KEYS);
   const int nq = nl / kThreads;
   Queues<KB> q;
-  KeyQueues<KB> kq;  // bf16 key path
+  KeyQueues<KB> kq;  // bf16 key path, k_b >= 2
+  PairQueues pq;     // bf16 key path, k_b = 1
   int st = 0;       // ring stage of the next tile
   uint32_t ph = 0;  // its full-barrier parity
   int64_t g = s0;
@@ -475,7 +543,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
     const uint32_t len = static_cast<uint32_t>(pend - g);  // < 2^31
     const uint32_t pos_thread = static_cast<uint32_t>(a) + 4u * tid;
-    if constexpr (KEYS)
+    if constexpr (KEYS && KB == 1)
+      pq.reset();
+    else if constexpr (KEYS)
       kq.reset();
     else
       q.reset();
@@ -487,7 +557,42 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
                                  !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
         const T* stage_tile = ring + static_cast<size_t>(st) * kTileElems;
-        if constexpr (KEYS) {
+        if constexpr (KEYS && KB == 1) {
+          // Slices of kTile elements as in the k_b >= 2 key path; a slice with
+          // a NaN or +-inf takes the element-wise update.
+          constexpr int U = kTile / kLanes;
+#pragma unroll
+          for (int h = 0; h < kTileElems / kTile; ++h) {
+            const uint32_t hoff = static_cast<uint32_t>(h * kTile);
+            const T* tile = stage_tile + hoff + 4 * tid;
+            const uint32_t ord0 = (done + hoff) / static_cast<uint32_t>(kLanes);
+            if (hoff + kTile <= c) {
+              uint2 w[U];
+#pragma unroll
+              for (int u = 0; u < U; ++u) w[u] = *reinterpret_cast<const uint2*>(tile + kLanes * u);
+              uint32_t mx = 0u, my = 0u;
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                mx = bf16x2_nonfinite_acc(w[u].x, mx);
+                my = bf16x2_nonfinite_acc(w[u].y, my);
+              }
+              if (!(bf16x2_has_nan(mx) | bf16x2_has_nan(my))) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) pq.offer4(w[u], ord0 + u);
+              } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u) pq.offer4_exact(w[u], ord0 + u);
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < U; ++u) {
+                const uint32_t off = hoff + 4u * tid + static_cast<uint32_t>(kLanes * u);
+                if (off < c)
+                  pq.offer4_exact(*reinterpret_cast<const uint2*>(tile + kLanes * u), ord0 + u);
+              }
+            }
+          }
+        } else if constexpr (KEYS) {
           // In slices of kTile elements: stripe u of a slice is queue ordinal
           // (done + hoff) / kLanes + u.  A pair NaN check per slice picks the
           // cheap or the NaN-aware codes.
@@ -580,7 +685,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
       group_sync(kThreads);
       if (*skip_flag) break;
     }
-    if constexpr (KEYS) {
+    if constexpr (KEYS && KB == 1) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) pq.store(v, lanebuf + static_cast<size_t>(4 * tid + v), pos_thread);
+    } else if constexpr (KEYS) {
       kq.combine();
 #pragma unroll
       for (int v = 0; v < 4; ++v)

@@ -500,13 +500,15 @@ def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(bits.astype(np.uint16).view(np.int16)).view(torch.bfloat16)
 
 
-@pytest.mark.parametrize("kb", [2, 3, 4])
+@pytest.mark.parametrize("kb", [1, 2, 3, 4])
 def test_bf16_key_queues_special_bits(oracle_mod, kb):
     """bf16 rows with k_b >= 2 run on 32-bit order keys (value code and queue
-    ordinal in one word).  Every special bit pattern must keep the total
-    order: NaNs of any sign and payload tie above +inf, -0 ties +0, -inf is
-    below every number, denormals order as numbers, equal values go by
-    index -- whole rows, split rows and ragged tails."""
+    ordinal in one word), k_b = 1 on packed bf16x2 queues.  Every special bit
+    pattern must keep the total order: NaNs of any sign and payload tie above
+    +inf, -0 ties +0, -inf is below every number, denormals order as numbers,
+    equal values go by index -- whole rows, split rows and ragged tails; and
+    with zeros and denormals only (no NaN or infinity), the packed compare of
+    the k_b = 1 fast path sees them too."""
     rng = np.random.default_rng(700 + kb)
     specials = np.array([0x7FC0, 0x7F81, 0xFFC1, 0x7FFF, 0xFF80, 0x7F80, 0x0000, 0x8000,
                          0x0001, 0x8001, 0x007F, 0x807F, 0x3F80, 0xBF80], np.uint16)
@@ -518,3 +520,10 @@ def test_bf16_key_queues_special_bits(oracle_mod, kb):
         bits[pick] = rng.choice(specials, size=int(pick.sum()))
         x = _bf16_from_bits(bits)
         _bf16_check(x, k, b, kb, oracle_mod)
+    finite = np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x807F], np.uint16)
+    for rows, n, k, b in [(6, 65536, 300, 256), (3, 400000, 700, 512)]:
+        bits = rng.integers(0x0000, 0x0100, size=(rows, n)).astype(np.uint16)  # denormals, ties
+        bits[rng.random((rows, n)) < 0.5] |= 0x8000
+        pick = rng.random((rows, n)) < 0.05
+        bits[pick] = rng.choice(finite, size=int(pick.sum()))
+        _bf16_check(_bf16_from_bits(bits), k, b, kb, oracle_mod)
