@@ -279,12 +279,12 @@ __device__ __forceinline__ bool bf16x2_has_nan(uint32_t w) {
   return ((w & 0x7FFFu) > 0x7F80u) | (((w >> 16) & 0x7FFFu) > 0x7F80u);
 }
 
-// k_b = 1 on bf16 rows: a thread's four queues (the float4 layout) as two
-// bf16x2 value words (queues 0, 1 and 2, 3) and two words of 16-bit stripe
-// ordinals (0xFFFF: empty), so that one packed compare and two bit-selects
-// update two queues.  A finite element replaces its queue's entry when it is
+// k_b <= 2 on bf16 rows: a thread's four queues (the float4 layout) as, per
+// slot, two bf16x2 value words (queues 0, 1 and 2, 3) and two words of 16-bit
+// stripe ordinals (0xFFFF: empty), so that packed compares and bit-selects
+// update two queues at once.  A finite element enters a slot when it is
 // strictly larger (ties keep the earlier stripe; -0 and +0 compare equal);
-// the entry starts at -inf, which every finite element beats.  A slice that
+// entries start at -inf, which every finite element beats.  A slice that
 // holds a NaN or +-inf takes the element-wise update under the total order
 // (16-bit order codes: NaN above +inf, -0 = +0, an empty queue takes anything).
 __device__ __forceinline__ uint32_t bf16x2_gt_mask(uint32_t a, uint32_t b) {
@@ -298,50 +298,84 @@ __device__ __forceinline__ uint32_t bf16_order_code(uint32_t h) {
   return (h & 0x8000u) ? ((h ^ 0xFFFFu) + 1u) & 0xFFFFu : (h ^ 0x8000u);
 }
 
+template <int KB>
 struct PairQueues {
-  uint32_t val[2], ord[2];
+  uint32_t val[KB][2], ord[KB][2];  // slot s of queues (0, 1) and (2, 3)
 
   __device__ __forceinline__ void reset() {
-    val[0] = val[1] = 0xFF80FF80u;  // -inf, -inf
-    ord[0] = ord[1] = 0xFFFFFFFFu;  // empty, empty
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      val[s][0] = val[s][1] = 0xFF80FF80u;  // -inf, -inf
+      ord[s][0] = ord[s][1] = 0xFFFFFFFFu;  // empty, empty
+    }
   }
 
   // Four consecutive finite bf16 (w.x: queues 0, 1; w.y: queues 2, 3) at
-  // stripe ordinal o.
+  // stripe ordinal o.  The slots are sorted, so x above slot s implies x
+  // above every later slot: slot s takes slot s-1 where x beats it, else x
+  // where x beats slot s, else keeps its entry.
   __device__ __forceinline__ void offer4(uint2 w, uint32_t o) {
     const uint32_t o2 = o * 0x00010001u;
-    const uint32_t m0 = bf16x2_gt_mask(w.x, val[0]);
-    const uint32_t m1 = bf16x2_gt_mask(w.y, val[1]);
-    val[0] = (w.x & m0) | (val[0] & ~m0);
-    ord[0] = (o2 & m0) | (ord[0] & ~m0);
-    val[1] = (w.y & m1) | (val[1] & ~m1);
-    ord[1] = (o2 & m1) | (ord[1] & ~m1);
+    const uint32_t xs[2] = {w.x, w.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t x = xs[i];
+      uint32_t m[KB];
+#pragma unroll
+      for (int s = 0; s < KB; ++s) m[s] = bf16x2_gt_mask(x, val[s][i]);
+#pragma unroll
+      for (int s = KB - 1; s >= 0; --s) {
+        const uint32_t tv = (x & m[s]) | (val[s][i] & ~m[s]);
+        const uint32_t to = (o2 & m[s]) | (ord[s][i] & ~m[s]);
+        if (s > 0) {
+          val[s][i] = (val[s - 1][i] & m[s - 1]) | (tv & ~m[s - 1]);
+          ord[s][i] = (ord[s - 1][i] & m[s - 1]) | (to & ~m[s - 1]);
+        } else {
+          val[s][i] = tv;
+          ord[s][i] = to;
+        }
+      }
+    }
   }
 
   __device__ __forceinline__ void offer4_exact(uint2 w, uint32_t o) {
     const uint32_t in[2] = {w.x, w.y};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int word = e >> 1, sh = (e & 1) * 16;
-      const uint32_t h = (in[word] >> sh) & 0xFFFFu;
-      const uint32_t cur = (val[word] >> sh) & 0xFFFFu;
-      const uint32_t co = (ord[word] >> sh) & 0xFFFFu;
-      if (co == 0xFFFFu || bf16_order_code(h) > bf16_order_code(cur)) {
-        val[word] = (val[word] & ~(0xFFFFu << sh)) | (h << sh);
-        ord[word] = (ord[word] & ~(0xFFFFu << sh)) | (o << sh);
+      const int i = e >> 1, sh = (e & 1) * 16;
+      const uint32_t lane_mask = 0xFFFFu << sh;
+      const uint32_t h = (in[i] >> sh) & 0xFFFFu;
+      // The first slot that is empty or holds a smaller entry takes the
+      // element; every later entry moves down one slot (the last drops out).
+      bool placed = false;
+      uint32_t mv = h, mo = o;  // the entry to write next (ordinal 0xFFFF: none)
+#pragma unroll
+      for (int s = 0; s < KB; ++s) {
+        const uint32_t cur = (val[s][i] >> sh) & 0xFFFFu;
+        const uint32_t co = (ord[s][i] >> sh) & 0xFFFFu;
+        if (!placed) placed = co == 0xFFFFu || bf16_order_code(h) > bf16_order_code(cur);
+        if (placed && mo != 0xFFFFu) {
+          val[s][i] = (val[s][i] & ~lane_mask) | (mv << sh);
+          ord[s][i] = (ord[s][i] & ~lane_mask) | (mo << sh);
+          mv = cur;
+          mo = co;
+        }
       }
     }
   }
 
-  // Queue v as one packed (order key, ~position) word, position = pos_thread
+  // Queue v as KB packed (order key, ~position) words, position = pos_thread
   // + v + ordinal * kLanes (0: empty).
   __device__ __forceinline__ void store(int v, uint64_t* dst, uint32_t pos_thread) const {
-    const int word = v >> 1, sh = (v & 1) * 16;
-    const uint32_t o = (ord[word] >> sh) & 0xFFFFu;
-    const uint32_t h = (val[word] >> sh) & 0xFFFFu;
-    dst[0] = o == 0xFFFFu ? 0ull
-                          : pack(order_key(__uint_as_float(h << 16)),
-                                 pos_thread + static_cast<uint32_t>(v) + o * static_cast<uint32_t>(kLanes));
+    const int i = v >> 1, sh = (v & 1) * 16;
+#pragma unroll
+    for (int s = 0; s < KB; ++s) {
+      const uint32_t o = (ord[s][i] >> sh) & 0xFFFFu;
+      const uint32_t h = (val[s][i] >> sh) & 0xFFFFu;
+      dst[s] = o == 0xFFFFu ? 0ull
+                            : pack(order_key(__uint_as_float(h << 16)),
+                                   pos_thread + static_cast<uint32_t>(v) + o * static_cast<uint32_t>(kLanes));
+    }
   }
 };
 
@@ -427,8 +461,11 @@ struct KeyQueues {
 #ifndef TOPK_BF16_KEYS
 #define TOPK_BF16_KEYS 1
 #endif
-#ifndef TOPK_BF16_KEYS_MIN_KB  // smallest k_b that takes the key path (k_b = 1: PairQueues)
+#ifndef TOPK_BF16_KEYS_MIN_KB  // smallest k_b that takes the key path
 #define TOPK_BF16_KEYS_MIN_KB 1
+#endif
+#ifndef TOPK_BF16_PAIR_MAX_KB  // largest k_b on packed bf16x2 queues (PairQueues)
+#define TOPK_BF16_PAIR_MAX_KB 2
 #endif
 
 #ifndef TOPK_SPARSE_MIN_KB  // smallest k_b that takes the survivor (sparse / wide) update
@@ -451,8 +488,8 @@ constexpr int kPipeThreads = kThreads + 32;  // consumers + one producer warp
 // the kThreads consumer threads never wait for each other inside a piece.
 // SAMPLE: the instantiation that also draws each row's token after Stage 2
 // (p.tail); without it the sampling code is not compiled in at all.
-// KEYS: bf16 rows on 16-bit codes -- k_b >= 2 in KeyQueues (see bf16 order
-// keys), k_b = 1 in PairQueues.
+// KEYS: bf16 rows on 16-bit codes -- k_b <= TOPK_BF16_PAIR_MAX_KB in
+// PairQueues, larger k_b in KeyQueues (see bf16 order keys).
 template <typename T, int KB, bool SAMPLE = false, bool KEYS = false>
 __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<T> p, int stages,
                                                                   int cand_cap, int layout) {
@@ -532,7 +569,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
   const int nq = nl / kThreads;
   Queues<KB> q;
   KeyQueues<KB> kq;  // bf16 key path, k_b >= 2
-  PairQueues pq;     // bf16 key path, k_b = 1
+  PairQueues<(KB <= 2 ? KB : 1)> pq;  // bf16 key path, packed queues
   int st = 0;       // ring stage of the next tile
   uint32_t ph = 0;  // its full-barrier parity
   int64_t g = s0;
@@ -543,7 +580,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
     const int64_t pend = (row0 + n < e0) ? row0 + n : e0;
     const uint32_t len = static_cast<uint32_t>(pend - g);  // < 2^31
     const uint32_t pos_thread = static_cast<uint32_t>(a) + 4u * tid;
-    if constexpr (KEYS && KB == 1)
+    if constexpr (KEYS && KB <= TOPK_BF16_PAIR_MAX_KB)
       pq.reset();
     else if constexpr (KEYS)
       kq.reset();
@@ -557,8 +594,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
                                  !*abort_flag && mbar_wait_or_abort(full + st, ph, abort_flag));
       if (ok) {
         const T* stage_tile = ring + static_cast<size_t>(st) * kTileElems;
-        if constexpr (KEYS && KB == 1) {
-          // Slices of kTile elements as in the k_b >= 2 key path; a slice with
+        if constexpr (KEYS && KB <= TOPK_BF16_PAIR_MAX_KB) {
+          // Slices of kTile elements as in the order-key path; a slice with
           // a NaN or +-inf takes the element-wise update.
           constexpr int U = kTile / kLanes;
 #pragma unroll
@@ -685,9 +722,10 @@ __global__ void __launch_bounds__(kPipeThreads, 2) bucket_select_tma(SelectArgs<
       group_sync(kThreads);
       if (*skip_flag) break;
     }
-    if constexpr (KEYS && KB == 1) {
+    if constexpr (KEYS && KB <= TOPK_BF16_PAIR_MAX_KB) {
 #pragma unroll
-      for (int v = 0; v < 4; ++v) pq.store(v, lanebuf + static_cast<size_t>(4 * tid + v), pos_thread);
+      for (int v = 0; v < 4; ++v)
+        pq.store(v, lanebuf + static_cast<size_t>(4 * tid + v) * KB, pos_thread);
     } else if constexpr (KEYS) {
       kq.combine();
 #pragma unroll

@@ -231,14 +231,15 @@ int plan_select_kb(bool fast, int64_t rows, int64_t n, int b, const DeviceInfo& 
   int per_sm = 0;
   const int64_t E = rows * n;
   if (fast) {
-    // bf16 rows (short enough for 16-bit queue ordinals): order-key queues
-    // (k_b >= 2) or packed bf16x2 queues (k_b = 1) in the float4 layout.  Otherwise k_b > 2 with b >= 512:
+    // bf16 rows (short enough for 16-bit queue ordinals): packed bf16x2 queues
+    // (k_b <= 2) or order-key queues (k_b > 2) in the float4 layout.  Otherwise k_b > 2 with b >= 512:
     // the 16-warp kernel, one lane per bucket (b lanes); smaller b keeps the
     // 8-warp kernel, whose 256 lanes split a bucket over fewer queues (fewer
     // inserts).
     constexpr bool kKeyType = sizeof(T) == 2 && KB >= TOPK_BF16_KEYS_MIN_KB;
-    // k_b = 1 keeps ordinal 0xFFFF for an empty queue: one stripe less.
-    const bool keys = kKeyType && TOPK_BF16_KEYS && n <= (KB == 1 ? kKeyMaxPiece - kLanes : kKeyMaxPiece);
+    // The packed queues keep ordinal 0xFFFF for an empty slot: one stripe less.
+    const bool keys = kKeyType && TOPK_BF16_KEYS &&
+                      n <= (KB <= TOPK_BF16_PAIR_MAX_KB ? kKeyMaxPiece - kLanes : kKeyMaxPiece);
     pl->keys = keys;
     const bool wide = !keys && KB >= TOPK_SPARSE_MIN_KB && TOPK_WIDE_SPARSE && b >= kWideConsumers;
     pl->wide_nq = wide ? (b > kWideConsumers ? b / kWideConsumers : 1) : 0;

@@ -502,13 +502,13 @@ def _bf16_from_bits(bits: np.ndarray) -> torch.Tensor:
 
 @pytest.mark.parametrize("kb", [1, 2, 3, 4])
 def test_bf16_key_queues_special_bits(oracle_mod, kb):
-    """bf16 rows with k_b >= 2 run on 32-bit order keys (value code and queue
-    ordinal in one word), k_b = 1 on packed bf16x2 queues.  Every special bit
+    """bf16 rows with k_b > 2 run on 32-bit order keys (value code and queue
+    ordinal in one word), k_b <= 2 on packed bf16x2 queues.  Every special bit
     pattern must keep the total order: NaNs of any sign and payload tie above
     +inf, -0 ties +0, -inf is below every number, denormals order as numbers,
     equal values go by index -- whole rows, split rows and ragged tails; and
     with zeros and denormals only (no NaN or infinity), the packed compare of
-    the k_b = 1 fast path sees them too."""
+    the k_b <= 2 fast path sees them too."""
     rng = np.random.default_rng(700 + kb)
     specials = np.array([0x7FC0, 0x7F81, 0xFFC1, 0x7FFF, 0xFF80, 0x7F80, 0x0000, 0x8000,
                          0x0001, 0x8001, 0x007F, 0x807F, 0x3F80, 0xBF80], np.uint16)
